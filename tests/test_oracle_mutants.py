@@ -1,0 +1,72 @@
+"""The oracle's pins must catch plausible mistakes in it.
+
+Each case plants one mistake (a dropped term, a wrong sign, index or
+comparison) in a temporary copy of the oracle's C source, builds it, and runs
+the pin tests against that copy: they must fail.  The real oracle source is
+never modified.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "fr_oracle.c")
+
+MUTANTS = {
+    "score_sign": ("cand[nc].score = score[k] + ((double)row[tok] - lse);",
+                   "cand[nc].score = score[k] - ((double)row[tok] - lse);"),
+    "lse_drops_max": ("return m + log(s);", "return log(s);"),
+    "lse_max_wrong_way": ("if ((double)x[v] > m) m = (double)x[v];", "if ((double)x[v] < m) m = (double)x[v];"),
+    "order_ascending": ("if (a->score != b->score) return a->score > b->score ? -1 : 1;",
+                        "if (a->score != b->score) return a->score < b->score ? -1 : 1;"),
+    "tie_parent_reversed": ("if (a->parent != b->parent) return a->parent < b->parent ? -1 : 1;",
+                            "if (a->parent != b->parent) return a->parent > b->parent ? -1 : 1;"),
+    "tie_token_reversed": ("return (a->token > b->token) - (a->token < b->token);",
+                           "return (a->token < b->token) - (a->token > b->token);"),
+    "live_off_by_one": ("int32_t nlive = (int32_t)(nc < K ? nc : K);",
+                        "int32_t nlive = (int32_t)(nc < K ? nc : K - 1);"),
+    "children_wrong_level": ("int32_t code = c->codes[i * c->depth + t];",
+                             "int32_t code = c->codes[i * c->depth + 0];"),
+    "prefix_from_own_slot": ("new_prefix[j * D + l] = (l < t) ? prefix[c->parent * D + l] : -1;",
+                             "new_prefix[j * D + l] = (l < t) ? prefix[j * D + l] : -1;"),
+    "keeps_last_duplicate": ("return (a->row > b->row) - (a->row < b->row);",
+                             "return (a->row < b->row) - (a->row > b->row);"),
+    "bf16_ties_away": ("if (lower > 0x8000u || (lower == 0x8000u && lsb)) upper += 0x10000u;",
+                       "if (lower >= 0x8000u) upper += 0x10000u;"),
+    "splitmix_shift": ("z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;",
+                       "z = (z ^ (z >> 28)) * 0x94D049BB133111EBULL;"),
+    "logit_offset": ("return (float)(u >> 40) * 0x1p-21f - 4.0f;",
+                     "return (float)(u >> 40) * 0x1p-21f - 3.0f;"),
+    "prefix_hash_seed": ("uint64_t h = 0x243F6A8885A308D3ULL;", "uint64_t h = 0;"),
+    "token_base_skips_level": ("for (int32_t i = 0; i < level; ++i) base += cfg->codebook[i];",
+                               "for (int32_t i = 1; i < level; ++i) base += cfg->codebook[i];"),
+}
+
+
+def _run_mutant(name, tmpdir):
+    find, repl = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(find) == 1, "mutation site not found exactly once: %s" % name
+    path = os.path.join(tmpdir, name + ".c")
+    with open(path, "w") as f:
+        f.write(src.replace(find, repl))
+    so = os.path.join(tmpdir, name + ".so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           "-D_POSIX_C_SOURCE=199309L", "-o", so, path, "-lm"])
+    env = dict(os.environ, FR_ORACLE_LIB=so)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode, r.stdout[-400:]
+
+
+def test_every_planted_mistake_is_caught():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 2)) as ex:
+            results = dict(zip(MUTANTS, ex.map(lambda n: _run_mutant(n, tmp), MUTANTS)))
+    survivors = {n: out for n, (rc, out) in results.items() if rc == 0}
+    assert not survivors, "pins missed planted mistakes: %s" % sorted(survivors)
