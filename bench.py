@@ -1,0 +1,385 @@
+"""Benchmark of the trie-constrained wide beam-search decode on B200.
+
+One benchmark step = one full decode of one batch of requests (depth beam
+steps + finalize) over a resident catalog trie, with every step's logits
+already in HBM when the timed region starts (they are produced beforehand by
+an untimed decode; each step has its own 1.9-5 GB buffer, far larger than the
+126 MB L2, so no step re-reads cached logits).
+
+Metric: constrained beam candidates per second, B*K*depth per decode, summed
+over ranks (requests shard across GPUs with no collective: weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config serving]
+    python bench.py --impl reference     # the CPU oracle on a bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from trie_constrained_beam_fr_b200 import synth  # noqa: E402
+
+METRIC = "constrained beam candidates/sec (B·K·steps/s) and logits HBM GB/s vs 8 TB/s"
+UNIT = "candidates/s"
+STREAM_KERNEL_SRC = os.path.join(ROOT, "trie_constrained_beam_fr_b200", "csrc", "fr_step.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="fr", choices=["fr", "reference"])
+    p.add_argument("--config", default="serving", choices=[k for k in synth.WORKLOADS if k != "tiny"])
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ref-requests", type=int, default=1, help="requests per reference-arm sample")
+    return p.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(STREAM_KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(config: str):
+    """Per-launch DRAM bytes of the streaming kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(config)
+    if not e or e.get("kernel_sha") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+
+
+def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, sids=None, cat=None):
+    import oracle
+
+    if sids is None:
+        sids = synth.workload_catalog(w)
+    if cat is None:
+        cat = oracle.Catalog(sids, w.codebook_sizes)
+    cfg = oracle.Config.from_workload(w, B=n_requests, b_offset=first_request)
+    t0 = time.perf_counter()
+    r = oracle.decode(cfg, cat)
+    wall = time.perf_counter() - t0
+    method = wall - r.gen_seconds
+    return {"candidates": n_requests * w.K * w.depth, "method_s": method, "gen_s": r.gen_seconds, "wall_s": wall}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    w = synth.WORKLOADS[args.config]
+    sids = synth.workload_catalog(w)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    for i in range(args.warmup):
+        oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat)
+    samples = [oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat)
+               for i in range(args.steps)]
+    cand = sum(s["candidates"] for s in samples)
+    secs = sum(s["method_s"] for s in samples)
+    value = cand / secs
+    sample = ("%d request(s) of %s per step (of B=%d), full decode, oracle time excluding its logits generation"
+              % (args.ref_requests, w.name, w.B))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "depth": w.depth, "V": w.V, "codes_per_level": w.C,
+                   "catalog": w.n_items, "logits": w.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from trie_constrained_beam_fr_b200 import fr
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = synth.WORKLOADS[args.config]
+    B, K, D, V = w.B, w.K, w.depth, w.V
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    elt = w.elt_size
+    b_offset = rank * B  # each rank decodes its own requests
+
+    sids_np = synth.workload_catalog(w)
+    sids = torch.from_numpy(sids_np).to(dev)
+    stream = torch.cuda.current_stream()
+
+    # catalog trie (off the per-decode path; timed on its own)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    trie = fr.fr_trie_build(sids, w.codebook_sizes, w.sid_base)  # warm (allocations, first launch)
+    fr.fr_trie_destroy(trie)
+    torch.cuda.synchronize()
+    e0.record()
+    trie = fr.fr_trie_build(sids, w.codebook_sizes, w.sid_base)
+    e1.record()
+    torch.cuda.synchronize()
+    trie_ms = e0.elapsed_time(e1)
+    levels = fr.fr_trie_level_sizes(trie)
+    beam = fr.fr_beam_init(trie, B, K, V, w.dtype)
+
+    # one untimed decode produces every step's logits (prefix-dependent)
+    bufs = [torch.empty((B, K, V), dtype=tdt, device=dev) for _ in range(D)]
+    rows = []
+    fr.fr_beam_reset(beam)
+    for t in range(D):
+        o = fr.fr_beam_outputs(beam, B, K, D)
+        rows.append(int(o["live"].sum().item()))
+        fr.fr_gen_hash_logits(w.seed, b_offset, B, K, V, bufs[t], w.dtype, prefix=o["prefix"], t=t, live=o["live"])
+        fr.fr_beam_step(beam, bufs[t])
+    out_sids = torch.empty((B, K, D), dtype=torch.int32, device=dev)
+    out_scores = torch.empty((B, K), dtype=torch.float32, device=dev)
+    out_items = torch.empty((B, K), dtype=torch.int32, device=dev)
+    fr.fr_beam_finalize(beam, out_sids, out_scores, out_items)
+    st = fr.fr_beam_status(beam)
+    if st != fr.FR_OK:
+        raise RuntimeError("decode failed: " + fr.fr_status_string(st))
+    bytes_per_decode = sum(r * V * elt for r in rows)
+
+    def decode():
+        fr.fr_beam_reset(beam)
+        for t in range(D):
+            fr.fr_beam_step(beam, bufs[t])
+        fr.fr_beam_finalize(beam, out_sids, out_scores, out_items)
+
+    for _ in range(args.warmup):
+        decode()
+    torch.cuda.synchronize()
+    fr.fr_beam_read_timing(beam)  # clear
+    fr.fr_beam_set_timing(beam, True)
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        t_start.record()
+        for _ in range(args.steps):
+            decode()
+        t_end.record()
+        torch.cuda.synchronize()
+    barrier()
+    fr.fr_beam_set_timing(beam, False)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    stream_ms, select_ms = fr.fr_beam_read_timing(beam)
+    st = fr.fr_beam_status(beam)
+    if st != fr.FR_OK:
+        raise RuntimeError("timed decode failed: " + fr.fr_status_string(st))
+    ms_per_decode = elapsed_ms / args.steps
+    cands_per_decode = B * K * D
+    value = world * cands_per_decode * args.steps / (elapsed_ms / 1e3)
+
+    # roofline of the dominant kernel: the streaming log-sum-exp / candidate kernel
+    peak, peak_kind = measured_peaks()
+    n_launch = len(stream_ms)
+    per_step_bytes = [r * V * elt for r in rows]
+    alg_bytes = sum(per_step_bytes[i % D] for i in range(n_launch))
+    stream_total_ms = float(np.sum(stream_ms))
+    achieved = alg_bytes / (stream_total_ms / 1e3) / 1e9
+    traffic = recorded_traffic(w.name)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "peak_source": peak_kind, "kernel": "k_stream",
+                "alg_bytes_per_launch": alg_bytes / max(1, n_launch),
+                "ms_per_launch": stream_total_ms / max(1, n_launch)}
+    per_step = []
+    for t in range(D):
+        sm = [stream_ms[i] for i in range(t, n_launch, D)]
+        se = [select_ms[i] for i in range(t, n_launch, D)]
+        per_step.append({"t": t, "live_rows": rows[t], "stream_us": 1e3 * float(np.mean(sm)),
+                         "select_us": 1e3 * float(np.mean(se)),
+                         "stream_gbs": per_step_bytes[t] / (float(np.mean(sm)) / 1e3) / 1e9})
+    hbm_gbs_decode = bytes_per_decode / (ms_per_decode / 1e3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        try:
+            for t in range(D):
+                h = torch.empty((B, K, V), dtype=tdt, pin_memory=True)
+                h.copy_(bufs[t])
+                host.append(h)
+        except RuntimeError:
+            host = [torch.empty((B, K, V), dtype=tdt, pin_memory=True).copy_(bufs[1 % D])] * D
+        h_sids = torch.empty((B, K, D), dtype=torch.int32, pin_memory=True)
+        h_scores = torch.empty((B, K), dtype=torch.float32, pin_memory=True)
+        h_items = torch.empty((B, K), dtype=torch.int32, pin_memory=True)
+
+        def e2e_decode():
+            fr.fr_beam_reset(beam)
+            for t in range(D):
+                bufs[t].copy_(host[t], non_blocking=True)
+                fr.fr_beam_step(beam, bufs[t])
+            fr.fr_beam_finalize(beam, out_sids, out_scores, out_items)
+            h_sids.copy_(out_sids, non_blocking=True)
+            h_scores.copy_(out_scores, non_blocking=True)
+            h_items.copy_(out_items, non_blocking=True)
+
+        e2e_decode()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.e2e_steps):
+            e2e_decode()
+        b_.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b_)) / args.e2e_steps
+        e2e = {"value": world * cands_per_decode / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": D * B * K * V * elt,
+               "d2h_bytes_per_step": B * K * D * 4 + B * K * 4 + B * K * 4,
+               "ms_per_step": e2e_ms, "steps": args.e2e_steps}
+        del host
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = oracle_sample(w, 1, first_request=0, sids=sids_np)
+        cpu = {"value": s["candidates"] / s["method_s"], "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "request 0 of %s (1 of B=%d), full decode, single-threaded C oracle in double, "
+                         "time excluding its logits generation (%.1f s method, %.1f s generation)"
+                         % (w.name, w.B, s["method_s"], s["gen_s"])}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B_per_gpu": B, "K": K, "depth": D, "V": V, "codes_per_level": w.C,
+                       "catalog": w.n_items, "logits": w.dtype, "trie_levels": levels,
+                       "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"
+                             % (B * K * V * elt / 1e9),
+                       "step": "one full decode: depth beam steps + finalize"},
+            "hbm_gbs": hbm_gbs_decode, "hbm_frac_of_8tbs": hbm_gbs_decode / 8000.0,
+            "roofline": roofline, "per_step": per_step, "trie_build_ms": trie_ms,
+            "gpu_launches": args.steps * (2 * D + 2),
+            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    fr.fr_beam_destroy(beam)
+    fr.fr_trie_destroy(trie)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+/*
+ * fr.h -- C ABI of libfr: the trie-constrained wide beam-search decode step
+ * of generative recommendation, as hand-written CUDA for B200 (sm_100a).
+ *
+ * What it computes ("flashrec 0.1.1 METADATA", opening section and
+ * §Features/Decoding; "beamgrad 2.0.0 PKG-INFO", first code example and
+ * §Features):  an item is a semantic ID (SID), a fixed-depth tuple of codes,
+ * one code per level; SID token of (level l, code c) is
+ * sid_base + C_0 + ... + C_{l-1} + c.  A request decodes `depth` steps at beam
+ * width K.  At step t every live beam's next-token logits row is normalised
+ * with log-softmax over the whole vocabulary V, only the children that the
+ * catalog trie allows under the beam's prefix become candidates (illegal SIDs
+ * are never candidates), each candidate's score is the beam's running score
+ * plus the child token's log-probability, and the K best candidates of the
+ * request survive under a strict total order: higher score first, then lower
+ * parent slot, then lower token.  Each survivor records its parent slot (for
+ * KV-cache reordering), its token and its trie node; fewer than K candidates
+ * leave the remaining slots dead.
+ *
+ * Conventions (all functions):
+ *  - Every device buffer passed in is owned by the caller and must stay valid
+ *    until the stream work that uses it completes.  Handles (fr_trie,
+ *    fr_beam) and everything they allocate are owned by the library.
+ *  - Calls taking a stream are stream-ordered and asynchronous unless stated;
+ *    they allocate nothing and never synchronise, so fr_beam_step and
+ *    fr_beam_finalize can be captured into a CUDA graph.
+ *  - Argument errors are returned at once, before any work is queued.
+ *    Errors found on the device (NaN/+inf logits, corrupt trie node ids, a
+ *    bounded wait that expired) are recorded in a sticky per-beam status word
+ *    and returned by fr_beam_status and by the synchronising calls.
+ *  - Limits: depth <= 16, every codebook size in [1, 65536], the packed SID
+ *    key sum_l ceil(log2 C_l) <= 63 bits, catalog size < 2^31, 1 <= K <= 1024,
+ *    1 <= B <= 4096, B*K*V < 2^53.
+ *  - Determinism: the same inputs on the same device give bit-identical
+ *    outputs (fixed reduction orders, no floating-point atomics).
+ */
+#ifndef FR_H
+#define FR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary-compatible with cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fr_stream;
+
+typedef enum {
+    FR_OK = 0,
+    FR_ERR_INVALID_ARG = 1,     /* bad size, pointer, limit or layout */
+    FR_ERR_DUPLICATE_SID = 2,   /* fr_trie_build with dedupe = 0 saw a repeated SID */
+    FR_ERR_CODE_RANGE = 3,      /* a code outside [0, C_l) */
+    FR_ERR_STATE = 4,           /* call out of order (e.g. more than depth steps) */
+    FR_ERR_CUDA = 5,            /* a CUDA runtime call failed */
+    FR_ERR_OOM = 6,             /* device allocation failed */
+    FR_ERR_NAN_LOGIT = 7,       /* a live row's log-sum-exp was not finite (NaN or +inf logits) */
+    FR_ERR_DEVICE = 8,          /* device-side consistency check failed (bad node id, expired wait) */
+    FR_ERR_NOT_IN_CATALOG = 9   /* fr_beam_set_state got a prefix that the trie does not hold */
+} fr_status;
+
+typedef enum { FR_F32 = 0, FR_BF16 = 1 } fr_dtype;
+
+typedef struct fr_trie fr_trie; /* opaque, library-owned */
+typedef struct fr_beam fr_beam; /* opaque, library-owned */
+
+const char* fr_status_string(fr_status s);
+
+/* ------------------------------------------------------------------------ */
+/* Catalog trie.  "flashrec 0.1.1 METADATA" §Features/Decoding: the catalog of
+ * valid SIDs is held as a CSR-sparse trie and restricts every continuation.
+ *
+ * Layout built on the device: level l (0..depth) holds the distinct length-l
+ * SID prefixes in lexicographic order (level 0 = the root alone, level depth
+ * = the distinct SIDs).  child_off[l][n] .. child_off[l][n+1] are the level-l+1
+ * children of level-l node n, sorted by code; code[l][m] is the last code of
+ * level-l node m; leaf_row[m] is the catalog row of SID m (the first row when
+ * the catalog repeats a SID).
+ *
+ * fr_trie_build:
+ *   sids_dev        device int32 [n, depth], row-major, codes (not tokens); read only
+ *   n               catalog rows, 1 <= n < 2^31
+ *   depth           SID depth D, 1..16
+ *   codebook_sizes  host int32 [depth], C_l in [1, 65536]
+ *   sid_base        token id of (level 0, code 0), >= 0
+ *   dedupe          1: repeated SIDs keep their first row; 0: FR_ERR_DUPLICATE_SID
+ *   stream          work is queued on it; the call synchronises it before returning
+ *   out             receives the handle (NULL on error)
+ * Returns FR_ERR_CODE_RANGE if any code is outside [0, C_l).
+ * The build is off the per-step path: it allocates and synchronises. */
+fr_status fr_trie_build(const int32_t* sids_dev, int64_t n, int32_t depth,
+                        const int32_t* codebook_sizes, int32_t sid_base, int32_t dedupe,
+                        fr_stream stream, fr_trie** out);
+
+/* nodes_per_level: host int64 [depth + 1], level 0 = 1 (the root). */
+fr_status fr_trie_level_sizes(const fr_trie* trie, int64_t* nodes_per_level);
+
+/* depth, sid_base, codebook sizes (host int32 [depth], may be NULL) and the
+ * largest child count of any node (bounds the candidates per beam). */
+fr_status fr_trie_info(const fr_trie* trie, int32_t* depth, int32_t* sid_base,
+                       int32_t* codebook_sizes, int32_t* max_fanout);
+
+/* Copies level l's CSR arrays to the host (synchronous; for tests and
+ * inspection).  child_off_host: int32 [nodes[l] + 1] for l < depth, else must
+ * be NULL; code_host: int32 [nodes[l]] for l >= 1, else must be NULL. */
+fr_status fr_trie_copy_level(const fr_trie* trie, int32_t level, int32_t* child_off_host,
+                             int32_t* code_host);
+
+/* leaf_rows_host: int32 [nodes[depth]] (synchronous). */
+fr_status fr_trie_copy_leaf_rows(const fr_trie* trie, int32_t* leaf_rows_host);
+
+void fr_trie_destroy(fr_trie* trie);
+
+/* ------------------------------------------------------------------------ */
+/* Beam search.  "beamgrad 2.0.0 PKG-INFO" first code example: the step gets
+ * next-token scores of shape [B, K, V] for every beam's prefix.
+ *
+ * fr_beam_init: B requests of K beams over a V-token vocabulary whose logits
+ * come as `dtype` (FR_F32 or FR_BF16).  The SID token range of `trie` must lie
+ * inside [0, V).  Every request starts from one live root beam (empty prefix,
+ * score 0, KV slot b*K); slots 1..K-1 are dead.  Allocates device state
+ * (synchronous); the handle keeps a pointer to `trie`, which must outlive it. */
+fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int32_t V, fr_dtype dtype,
+                       fr_stream stream, fr_beam** out);
+
+/* Back to the initial state (root beams, step 0, status cleared); async. */
+fr_status fr_beam_reset(fr_beam* beam, fr_stream stream);
+
+/* One decode step (async).  logits_dev: device [B, K, V] of the beam's dtype,
+ * row (b, k) at logits_dev + (b*K + k)*ld elements, ld >= V, aligned to the
+ * element size.  Only the rows of live beams are read.  Returns FR_ERR_STATE
+ * after `depth` steps.  The step's results are visible through
+ * fr_beam_outputs once the stream reaches them. */
+fr_status fr_beam_step(fr_beam* beam, const void* logits_dev, int64_t ld, fr_stream stream);
+
+/* Device views of the latest step's results, valid until the next
+ * fr_beam_step / fr_beam_reset / fr_beam_set_state.  Any out-pointer may be
+ * NULL.  All [B, K] row-major, slot j of request b at b*K + j, rank order:
+ *   parent   int32  slot of the parent beam in the previous step (-1 dead)
+ *   token    int32  token chosen at this step (-1 dead)
+ *   node     int32  trie node id at level = steps done (-1 dead)
+ *   score    float  running score, sum of log-probabilities (-inf dead)
+ *   kv_slot  int32  the parent's KV slot carried forward (-1 dead)
+ *   live     int32  [B] live beams per request
+ *   prefix   int32  [B, K, depth] SID tokens so far (-1 beyond) */
+fr_status fr_beam_outputs(const fr_beam* beam, const int32_t** parent, const int32_t** token,
+                          const int32_t** node, const float** score, const int32_t** kv_slot,
+                          const int32_t** live, const int32_t** prefix);
+
+/* Steps done so far (0..depth). */
+int32_t fr_beam_steps_done(const fr_beam* beam);
+
+/* After `depth` steps (else FR_ERR_STATE): writes the ranked beams (async).
+ *   sids_dev    device int32 [B, K, depth] codes (-1 for dead beams)
+ *   scores_dev  device float [B, K] (-inf dead)
+ *   items_dev   device int32 [B, K] catalog row of each SID (-1 dead), or NULL */
+fr_status fr_beam_finalize(fr_beam* beam, int32_t* sids_dev, float* scores_dev, int32_t* items_dev,
+                           fr_stream stream);
+
+/* Synchronises the beam's last stream and returns its sticky device status
+ * (FR_OK, FR_ERR_NAN_LOGIT, FR_ERR_DEVICE, FR_ERR_NOT_IN_CATALOG) or FR_ERR_CUDA. */
+fr_status fr_beam_status(fr_beam* beam);
+
+/* Checkpoint / test hook (synchronous, host buffers).  get_state copies the
+ * current state out; set_state replaces it with `steps_done` steps taken:
+ *   live_host     int32 [B]
+ *   prefix_host   int32 [B, K, depth] codes (levels >= steps_done ignored)
+ *   score_host    float [B, K]
+ *   kv_host       int32 [B, K] or NULL (set_state: keep b*K + k)
+ *   node_host     int32 [B, K] (get_state only, may be NULL)
+ * set_state locates each live prefix in the trie on the device and returns
+ * FR_ERR_NOT_IN_CATALOG if one is missing. */
+fr_status fr_beam_get_state(fr_beam* beam, int32_t* steps_done, int32_t* live_host,
+                            int32_t* prefix_host, float* score_host, int32_t* kv_host,
+                            int32_t* node_host);
+fr_status fr_beam_set_state(fr_beam* beam, int32_t steps_done, const int32_t* live_host,
+                            const int32_t* prefix_host, const float* score_host,
+                            const int32_t* kv_host, fr_stream stream);
+
+/* Optional kernel timing.  While enabled, every fr_beam_step records CUDA
+ * events around its two kernels on the step's stream.  fr_beam_read_timing
+ * synchronises, returns up to max_steps per-step durations in milliseconds
+ * (stream_ms: the fused log-sum-exp / candidate kernel, select_ms: the top-K
+ * and reorder kernel) in step order, stores the count in *n, and clears. */
+fr_status fr_beam_set_timing(fr_beam* beam, int32_t enable);
+fr_status fr_beam_read_timing(fr_beam* beam, float* stream_ms, float* select_ms, int32_t max_steps,
+                              int32_t* n);
+
+void fr_beam_destroy(fr_beam* beam);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FR_H */

@@ -91,11 +91,11 @@ def lib():
         L.orc_step.restype = ctypes.c_int32
         L.orc_step.argtypes = [P(_Cfg), ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                P(ctypes.c_int32), P(ctypes.c_double), P(ctypes.c_int32), P(ctypes.c_double),
-                               P(ctypes.c_int32), P(ctypes.c_int32)]
+                               P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double)]
         L.orc_decode.restype = ctypes.c_int
         L.orc_decode.argtypes = [P(_Cfg), ctypes.c_void_p, P(ctypes.c_int32), P(ctypes.c_double),
                                  P(ctypes.c_int64), P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double),
-                                 P(ctypes.c_int32), P(ctypes.c_int32)]
+                                 P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double)]
         L.orc_gen_seconds.restype = ctypes.c_double
         L.orc_gen_seconds.argtypes = [ctypes.c_int32]
     return _lib
@@ -223,6 +223,7 @@ class StepResult:
     score: np.ndarray    # [K] float64
     parent: np.ndarray   # [K]
     token: np.ndarray    # [K]
+    excluded_best: float  # best candidate score that did not survive (-inf if none)
 
 
 def step(cfg: Config, cat: Catalog, b: int, t: int, live: int, prefix: np.ndarray,
@@ -235,13 +236,14 @@ def step(cfg: Config, cat: Catalog, b: int, t: int, live: int, prefix: np.ndarra
     nsc = np.empty(K, dtype=np.float64)
     par = np.empty(K, dtype=np.int32)
     tok = np.empty(K, dtype=np.int32)
+    exc = ctypes.c_double()
     c = cfg.c()
     nl = lib().orc_step(ctypes.byref(c), cat.handle, b, t, live, _ptr(pre, ctypes.c_int32), _ptr(sc, ctypes.c_double),
                         _ptr(npre, ctypes.c_int32), _ptr(nsc, ctypes.c_double), _ptr(par, ctypes.c_int32),
-                        _ptr(tok, ctypes.c_int32))
+                        _ptr(tok, ctypes.c_int32), ctypes.byref(exc))
     if nl < 0:
         raise ValueError("oracle step rejected its arguments")
-    return StepResult(int(nl), npre, nsc, par, tok)
+    return StepResult(int(nl), npre, nsc, par, tok, float(exc.value))
 
 
 @dataclass
@@ -254,6 +256,7 @@ class DecodeResult:
     step_score: np.ndarray    # [D, B, K]
     step_live: np.ndarray     # [D, B]
     step_prefix: np.ndarray   # [D, B, K, D]
+    step_excluded: np.ndarray  # [D, B] best non-surviving candidate score (-inf if none)
     gen_seconds: float = 0.0
 
 
@@ -267,12 +270,14 @@ def decode(cfg: Config, cat: Catalog) -> DecodeResult:
     ss = np.empty((D, B, K), dtype=np.float64)
     sl = np.empty((D, B), dtype=np.int32)
     spre = np.empty((D, B, K, D), dtype=np.int32)
+    sexc = np.empty((D, B), dtype=np.float64)
     c = cfg.c()
     lib().orc_gen_seconds(1)
     rc = lib().orc_decode(ctypes.byref(c), cat.handle, _ptr(sids, ctypes.c_int32), _ptr(scores, ctypes.c_double),
                           _ptr(items, ctypes.c_int64), _ptr(sp, ctypes.c_int32), _ptr(st, ctypes.c_int32),
-                          _ptr(ss, ctypes.c_double), _ptr(sl, ctypes.c_int32), _ptr(spre, ctypes.c_int32))
+                          _ptr(ss, ctypes.c_double), _ptr(sl, ctypes.c_int32), _ptr(spre, ctypes.c_int32),
+                          _ptr(sexc, ctypes.c_double))
     if rc != 0:
         raise ValueError("oracle decode failed: %s" % ERR_NAMES.get(rc, rc))
     gen = float(lib().orc_gen_seconds(1))
-    return DecodeResult(sids, scores, items, sp, st, ss, sl, spre, gen)
+    return DecodeResult(sids, scores, items, sp, st, ss, sl, spre, sexc, gen)

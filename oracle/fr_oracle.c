@@ -307,10 +307,12 @@ static double now_seconds(void) {
  *   score:       [K] running score of each live beam
  * Outputs (all [K], slots >= new live are dead: parent/token/code -1, score -inf):
  *   new_prefix   [K, depth], new_score [K], parent [K], token [K]
+ *   excluded_best  (may be NULL) score of the best candidate that did not
+ *                  survive, -inf if every candidate survived
  * Returns the new live count, or -1 on error. */
 int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t t, int32_t live,
                  const int32_t* prefix, const double* score, int32_t* new_prefix, double* new_score,
-                 int32_t* parent, int32_t* token) {
+                 int32_t* parent, int32_t* token, double* excluded_best) {
     const int32_t K = cfg->K, D = cfg->depth;
     if (t < 0 || t >= D || live < 0 || live > K) return -1;
     float* row = (float*)malloc(sizeof(float) * (size_t)cfg->V);
@@ -338,6 +340,7 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     }
     qsort(cand, (size_t)nc, sizeof(orc_cand), cmp_cand);
     int32_t nlive = (int32_t)(nc < K ? nc : K);
+    if (excluded_best) *excluded_best = (nc > nlive) ? cand[nlive].score : -INFINITY;
     for (int32_t j = 0; j < K; ++j) {
         if (j < nlive) {
             const orc_cand* c = &cand[j];
@@ -365,11 +368,13 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
  *   sids   [B, K, depth] codes (-1 for dead beams), scores [B, K] (-inf dead),
  *   items  [B, K] catalog row of each final SID (-1 dead),
  *   step_parent / step_token [depth, B, K], step_score [depth, B, K],
- *   step_live [depth, B]   (state after each step).
+ *   step_live [depth, B]   (state after each step),
+ *   step_prefix [depth, B, K, depth] and step_excluded [depth, B] (optional).
  * Returns ORC_OK or an error. */
 int orc_decode(const orc_cfg* cfg, const orc_catalog* cat, int32_t* sids, double* scores, int64_t* items,
                int32_t* step_parent, int32_t* step_token, double* step_score, int32_t* step_live,
-               int32_t* step_prefix /* [depth, B, K, depth] or NULL */) {
+               int32_t* step_prefix /* [depth, B, K, depth] or NULL */,
+               double* step_excluded /* [depth, B] or NULL */) {
     const int32_t B = cfg->B, K = cfg->K, D = cfg->depth;
     int32_t* pre = (int32_t*)malloc(sizeof(int32_t) * (size_t)K * D);
     int32_t* npre = (int32_t*)malloc(sizeof(int32_t) * (size_t)K * D);
@@ -384,7 +389,8 @@ int orc_decode(const orc_cfg* cfg, const orc_catalog* cat, int32_t* sids, double
         for (int32_t t = 0; t < D; ++t) {
             int32_t* par = step_parent + ((int64_t)t * B + b) * K;
             int32_t* tok = step_token + ((int64_t)t * B + b) * K;
-            live = orc_step(cfg, cat, b, t, live, pre, sc, npre, nsc, par, tok);
+            live = orc_step(cfg, cat, b, t, live, pre, sc, npre, nsc, par, tok,
+                            step_excluded ? step_excluded + (int64_t)t * B + b : NULL);
             if (live < 0) {
                 free(pre); free(npre); free(sc); free(nsc);
                 return ORC_ERR_ARG;

@@ -1,0 +1,71 @@
+"""Full-size workloads, in the launch configuration the benchmark times.
+
+For each catalog-scale workload the GPU decodes all B requests.  Every request
+is checked for the invariants (SIDs in the catalog, scores non-increasing,
+distinct beams, dead slots marked).  Sampled requests -- requests are
+independent, so the oracle decodes them one at a time -- are checked step by
+step under teacher forcing: the full batch is set to the GPU's own state except
+the sampled requests, which get the oracle's state, and one GPU step must then
+match the oracle's next step under the near-tie protocol."""
+import numpy as np
+import pytest
+
+import oracle
+from trie_constrained_beam_fr_b200 import synth
+
+from frlib import GpuBeam, check_invariants, compare_step, near_tie_in, oracle_cfg
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.mark.parametrize("name", ["serving", "wide_deep", "narrow", "skewed"])
+def test_full_size_workload(name):
+    w = synth.WORKLOADS[name]
+    sids = synth.workload_catalog(w)
+    samples = [0, w.B - 1]
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    refs = {b: oracle.decode(oracle_cfg(w, B=1, b_offset=b), cat) for b in samples}
+    gpu = GpuBeam(w, sids)
+    try:
+        views = gpu.decode()
+        g_sids, g_scores, g_items = gpu.finalize()
+        check_invariants(w, sids, g_sids, g_scores, g_items, views[-1].live)
+
+        # free running, sampled requests
+        for b in samples:
+            r = refs[b]
+            for t in range(w.depth):
+                p = compare_step(views[t].live[b], views[t].parent[b], views[t].token[b], views[t].score[b],
+                                 r.step_live[t, 0], r.step_parent[t, 0], r.step_token[t, 0], r.step_score[t, 0],
+                                 r.step_excluded[t, 0], where="free t=%d b=%d" % (t, b))
+                if p:
+                    assert near_tie_in(r.step_score[t, 0], r.step_live[t, 0], r.step_excluded[t, 0]), p
+                    break
+
+        # teacher forced, sampled requests, full batch
+        problems = []
+        for t in range(w.depth):
+            if t == 0:
+                live = np.ones(w.B, np.int32)
+                prefix = np.full((w.B, w.K, w.depth), -1, np.int32)
+                score = np.full((w.B, w.K), -np.inf, np.float32)
+                score[:, 0] = 0
+            else:
+                live = views[t - 1].live.copy()
+                prefix = views[t - 1].prefix.copy()
+                score = views[t - 1].score.copy()
+                for b in samples:
+                    r = refs[b]
+                    live[b] = r.step_live[t - 1, 0]
+                    prefix[b] = r.step_prefix[t - 1, 0]
+                    score[b] = r.step_score[t - 1, 0].astype(np.float32)
+            assert gpu.set_state(t, live, prefix, score) == 0
+            v = gpu.step(t)
+            for b in samples:
+                r = refs[b]
+                problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], r.step_live[t, 0],
+                                         r.step_parent[t, 0], r.step_token[t, 0], r.step_score[t, 0],
+                                         r.step_excluded[t, 0], where="forced t=%d b=%d" % (t, b))
+        assert not problems, "\n".join(problems[:20])
+    finally:
+        gpu.close()

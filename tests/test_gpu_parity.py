@@ -1,0 +1,219 @@
+"""CUDA beam step vs the oracle on small workloads (seconds for the oracle) that
+still span many CTAs, rows split across CTAs, ragged tails and the degenerate
+cases of the method.  Integer results (parents, tokens, nodes, SIDs, catalog
+rows) must be identical wherever the oracle's scores are separated by more than
+1e-4; scores must agree within 1e-4 (fp32 accumulation against double)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from trie_constrained_beam_fr_b200 import synth
+
+from frlib import GpuBeam, check_invariants, compare_step, near_tie_in, oracle_cfg
+
+pytestmark = pytest.mark.gpu
+
+W = synth.Workload
+SMALL = {
+    # the tiny workload itself
+    "tiny": synth.WORKLOADS["tiny"],
+    # bf16, V not a multiple of 8, SID range not 16-byte aligned, 3 requests
+    "ragged_bf16": W("ragged_bf16", B=3, K=16, depth=3, C=16, V=1003, sid_base=13, n_items=2000, dtype="bf16",
+                     seed=11, catalog_seed=11),
+    # rows of 20000 spread over ~1.7 CTAs each: cross-CTA partials
+    "mid_bf16": W("mid_bf16", B=4, K=64, depth=3, C=64, V=20000, sid_base=1000, n_items=20000, dtype="bf16",
+                  seed=2, catalog_seed=2),
+    "mid_f32_deep": W("mid_f32_deep", B=3, K=128, depth=4, C=32, V=9000, sid_base=100, n_items=60000, dtype="f32",
+                      seed=3, catalog_seed=3),
+    # full vocabulary, very few rows: a row split over ~74 CTAs at step 0
+    "full_vocab_few_rows": W("full_vocab_few_rows", B=2, K=4, depth=3, C=256, V=151936, sid_base=131072,
+                             n_items=5000, dtype="bf16", seed=4, catalog_seed=4),
+    "k1024": W("k1024", B=1, K=1024, depth=3, C=64, V=4096, sid_base=0, n_items=50000, dtype="f32", seed=5,
+               catalog_seed=5),
+    "greedy": W("greedy", B=2, K=1, depth=4, C=32, V=2000, sid_base=500, n_items=3000, dtype="bf16", seed=6,
+                catalog_seed=6),
+    "k_exceeds_catalog": W("k_exceeds_catalog", B=2, K=64, depth=3, C=16, V=64, sid_base=16, n_items=20,
+                           dtype="f32", seed=7, catalog_seed=7),
+    "skewed_small": W("skewed_small", B=2, K=128, depth=3, C=256, V=5000, sid_base=1000, n_items=30000,
+                      dtype="f32", seed=8, catalog_seed=8, zipf_levels=2),
+}
+
+
+def _catalog(w):
+    return synth.workload_catalog(w)
+
+
+def _teacher_forced(w, sids, gpu, ref):
+    """Step t of the GPU from the oracle's state after step t-1."""
+    problems = []
+    B, K, D = w.B, w.K, w.depth
+    for t in range(D):
+        if t == 0:
+            live = np.ones(B, np.int32)
+            prefix = np.full((B, K, D), -1, np.int32)
+            score = np.full((B, K), -np.inf, np.float32)
+            score[:, 0] = 0.0
+        else:
+            live = ref.step_live[t - 1].astype(np.int32)
+            prefix = ref.step_prefix[t - 1]
+            score = ref.step_score[t - 1].astype(np.float32)
+        assert gpu.set_state(t, live, prefix, score) == 0
+        v = gpu.step(t)
+        for b in range(B):
+            problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], ref.step_live[t, b],
+                                     ref.step_parent[t, b], ref.step_token[t, b], ref.step_score[t, b],
+                                     ref.step_excluded[t, b], where="t=%d b=%d" % (t, b))
+            # the node ids name the same prefixes: compare prefixes (codes)
+            n = int(ref.step_live[t, b])
+            sep = [j for j in range(n) if (j == 0 or ref.step_score[t, b, j - 1] - ref.step_score[t, b, j] > 1e-4)
+                   and (j == n - 1 or ref.step_score[t, b, j] - ref.step_score[t, b, j + 1] > 1e-4)]
+            if sep:
+                np.testing.assert_array_equal(v.prefix[b, sep, : t + 1], ref.step_prefix[t, b, sep, : t + 1])
+    return problems
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_teacher_forced_steps(name):
+    w = SMALL[name]
+    sids = _catalog(w)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    ref = oracle.decode(oracle_cfg(w), cat)
+    gpu = GpuBeam(w, sids)
+    try:
+        problems = _teacher_forced(w, sids, gpu, ref)
+    finally:
+        gpu.close()
+    assert not problems, "\n".join(problems[:20])
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_free_running_decode(name):
+    w = SMALL[name]
+    sids = _catalog(w)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    ref = oracle.decode(oracle_cfg(w), cat)
+    gpu = GpuBeam(w, sids)
+    try:
+        views = gpu.decode()
+        g_sids, g_scores, g_items = gpu.finalize()
+    finally:
+        gpu.close()
+    check_invariants(w, sids, g_sids, g_scores, g_items, views[-1].live)
+    for b in range(w.B):
+        diverged = False
+        for t in range(w.depth):
+            p = compare_step(views[t].live[b], views[t].parent[b], views[t].token[b], views[t].score[b],
+                             ref.step_live[t, b], ref.step_parent[t, b], ref.step_token[t, b],
+                             ref.step_score[t, b], ref.step_excluded[t, b], where="t=%d b=%d" % (t, b))
+            if p:
+                # allowed only at a documented near-tie; later steps then differ
+                assert near_tie_in(ref.step_score[t, b], ref.step_live[t, b], ref.step_excluded[t, b]), p
+                diverged = True
+                break
+        if not diverged:
+            n = int(ref.step_live[-1, b])
+            np.testing.assert_allclose(g_scores[b, :n], ref.scores[b, :n], atol=1e-4, rtol=0)
+            s = ref.scores[b]
+            for j in range(n):
+                if (j == 0 or s[j - 1] - s[j] > 1e-4) and (j == n - 1 or s[j] - s[j + 1] > 1e-4):
+                    np.testing.assert_array_equal(g_sids[b, j], ref.sids[b, j])
+                    assert g_items[b, j] == ref.items[b, j]
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid_bf16", "full_vocab_few_rows", "k_exceeds_catalog"])
+def test_all_equal_logits_closed_form(name):
+    """Every log-prob is -ln V: ranking is pure tie-breaking, so the beams are
+    the first K SIDs in lexicographic order, with score -D ln V."""
+    w = SMALL[name]
+    sids = _catalog(w)
+    ordered = np.unique(sids, axis=0)
+    gpu = GpuBeam(w, sids)
+    try:
+        views = gpu.decode(const=0.0)
+        g_sids, g_scores, g_items = gpu.finalize()
+    finally:
+        gpu.close()
+    n = min(w.K, ordered.shape[0])
+    for b in range(w.B):
+        assert views[-1].live[b] == n
+        np.testing.assert_array_equal(g_sids[b, :n], ordered[:n])
+        np.testing.assert_allclose(g_scores[b, :n], -w.depth * math.log(w.V), atol=1e-4, rtol=0)
+    # and the oracle agrees with the closed form on the same input
+    ref = oracle.decode(oracle_cfg(w, const=0.0), oracle.Catalog(sids, w.codebook_sizes))
+    np.testing.assert_array_equal(ref.sids[0, :n], ordered[:n])
+
+
+def test_single_child_chain_trie():
+    w = W("chain", B=2, K=8, depth=3, C=16, V=64, sid_base=16, n_items=5, dtype="f32", seed=9)
+    sids = np.array([[c, (c + 3) % 16, (c * 5) % 16] for c in range(5)], np.int32)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    ref = oracle.decode(oracle_cfg(w), cat)
+    gpu = GpuBeam(w, sids)
+    try:
+        views = gpu.decode()
+        g_sids, g_scores, g_items = gpu.finalize()
+    finally:
+        gpu.close()
+    for b in range(w.B):
+        assert views[-1].live[b] == 5
+        np.testing.assert_allclose(g_scores[b, :5], ref.scores[b, :5], atol=1e-4)
+        np.testing.assert_array_equal(g_sids[b], ref.sids[b])
+        np.testing.assert_array_equal(g_items[b], ref.items[b])
+
+
+@pytest.mark.parametrize("misalign,ld_pad", [(1, 0), (0, 5), (3, 7)])
+def test_strided_and_unaligned_rows(misalign, ld_pad):
+    w = SMALL["ragged_bf16"]
+    sids = _catalog(w)
+    ref = oracle.decode(oracle_cfg(w), oracle.Catalog(sids, w.codebook_sizes))
+    gpu = GpuBeam(w, sids, ld=w.V + ld_pad, misalign=misalign)
+    try:
+        views = gpu.decode()
+    finally:
+        gpu.close()
+    for b in range(w.B):
+        for t in range(w.depth):
+            p = compare_step(views[t].live[b], views[t].parent[b], views[t].token[b], views[t].score[b],
+                             ref.step_live[t, b], ref.step_parent[t, b], ref.step_token[t, b],
+                             ref.step_score[t, b], ref.step_excluded[t, b])
+            if p:
+                assert near_tie_in(ref.step_score[t, b], ref.step_live[t, b], ref.step_excluded[t, b]), p
+                break
+
+
+def test_deterministic_and_reset():
+    w = SMALL["mid_bf16"]
+    sids = _catalog(w)
+    gpu = GpuBeam(w, sids)
+    try:
+        a = gpu.decode()
+        fa = gpu.finalize()
+        b = gpu.decode()
+        fb = gpu.finalize()
+    finally:
+        gpu.close()
+    for x, y in zip(fa, fb):
+        np.testing.assert_array_equal(x, y)
+    for va, vb in zip(a, b):
+        np.testing.assert_array_equal(va.score.view(np.uint32), vb.score.view(np.uint32))
+        np.testing.assert_array_equal(va.parent, vb.parent)
+
+
+def test_kv_slots_follow_parents():
+    w = SMALL["ragged_bf16"]
+    sids = _catalog(w)
+    gpu = GpuBeam(w, sids)
+    try:
+        views = gpu.decode()
+    finally:
+        gpu.close()
+    prev_kv = np.full((w.B, w.K), -1, np.int32)
+    prev_kv[:, 0] = np.arange(w.B) * w.K
+    for v in views:
+        for b in range(w.B):
+            n = int(v.live[b])
+            np.testing.assert_array_equal(v.kv[b, :n], prev_kv[b, v.parent[b, :n]])
+            assert np.all(v.kv[b, n:] == -1)
+        prev_kv = v.kv

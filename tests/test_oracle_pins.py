@@ -275,6 +275,17 @@ def test_invariants_and_step_chaining():
                     assert st.token[j] == cfg.token_base(t) + st.prefix[j, t]
                     assert st.score[j] <= score[p]
                 assert np.all(st.parent[st.live:] == -1) and np.all(np.isneginf(st.score[st.live:]))
+                # the best excluded candidate is what a beam one wider keeps last
+                wider = oracle.Config(**{**cfg.__dict__, "K": K + 1})
+                pre1 = np.full((K + 1, cfg.depth), -1, np.int32)
+                pre1[:K] = prefix
+                sc1 = np.full(K + 1, -np.inf)
+                sc1[:K] = score
+                st1 = oracle.step(wider, cat, b, t, live, pre1, sc1)
+                if st1.live > st.live:
+                    assert st.excluded_best == st1.score[K]
+                else:
+                    assert np.isneginf(st.excluded_best)
                 prefix, score, live = st.prefix, st.score, st.live
             for j in range(live):
                 assert tuple(res.sids[b, j]) in catalog

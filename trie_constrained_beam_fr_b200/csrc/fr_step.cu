@@ -1,0 +1,863 @@
+// fr_step.cu -- the trie-constrained beam-search step on sm_100a.
+//
+// One step ("beamgrad 2.0.0 PKG-INFO", first code example and §Features;
+// "flashrec 0.1.1 METADATA", §Features/Decoding) is two kernels:
+//
+//  k_stream  log-sum-exp of every live logits row over the full vocabulary,
+//            then, for each row, the trie children's candidate scores
+//            score_k + (x[token] - lse_k).  HBM-bound: the live rows are read
+//            exactly once.  Persistent grid, one CTA per SM.  The flat element
+//            space of all live rows (request-major) is cut into equal,
+//            1024-element-aligned ranges, one per CTA, so every CTA streams
+//            the same number of bytes whatever the row count.  Inside a CTA
+//            one producer lane moves 32 KB chunks from HBM into a 6-stage
+//            shared-memory ring with 1-D bulk async copies completing on
+//            mbarriers; 16 consumer warps each reduce a 2 KB slice of every
+//            chunk (running max + scaled exp2 sum per lane).  At the end of a
+//            row segment the last consumer warp to arrive combines the 16
+//            warp partials in a fixed order and finishes the row; a row split
+//            across CTAs is finished by the last CTA to arrive (atomic
+//            counter, no waiting) from the per-CTA partials in CTA order.
+//            Ragged heads/tails that are not 16-byte aligned use plain loads.
+//
+//  k_select  per request: exact top-K of all its candidates under the strict
+//            order (score desc, slot asc) -- slot order is (parent slot,
+//            token) order -- by radix selection of order-preserving 32-bit
+//            keys (12-bit digits after skipping the bits all keys share),
+//            then a bitonic sort of the K winners on (key, ~slot); then the
+//            reorder gathers: backpointer, token, trie node, score, prefix and
+//            KV slot of every survivor, and the next step's candidate offsets.
+//
+// Every wait on an mbarrier is bounded: after 2 s the kernel records
+// FR_ERR_DEVICE in the beam's status word and returns.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fr_step.cuh"
+
+namespace fr {
+namespace {
+
+constexpr int NCW = 16;  // consumer warps
+constexpr int STREAM_THREADS = (NCW + 1) * 32;
+constexpr int STAGES = 6;
+constexpr int STAGE_BYTES = 32768;
+constexpr int VEC_PER_STAGE = STAGE_BYTES / 16;
+constexpr int VPL = VEC_PER_STAGE / (NCW * 32);  // 16-byte vectors per lane per chunk
+constexpr int64_t GRAN = 1024;                   // CTA ranges start at multiples of this many elements
+constexpr float L2E = 1.4426950408889634f;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
+
+struct SmemHdr {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    float2 part[STAGES][NCW];
+    int32_t segcnt[STAGES];
+    int32_t abort_flag;
+    int32_t pad;
+};
+
+struct StreamArgs {
+    const char* logits;
+    int64_t ld;
+    int32_t V, B, K, t, elt;
+    const int32_t* live;
+    const int32_t* node;
+    const float* score;
+    const int32_t* cand_off;
+    TrieDev trie;
+    float* cand;
+    int64_t cand_stride;
+    float2* partial;
+    int32_t* row_cnt;
+    int32_t* err;
+};
+
+struct Seg {
+    const char* ptr;     // row start
+    int64_t c0, c1;      // this CTA's element range in the row
+    int64_t a0, a1;      // 16-byte aligned interior of [c0, c1)
+    int32_t b, k;
+    int32_t nchunks;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
+                                         int32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            set_error(err, FR_ERR_DEVICE);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (draining copies in flight).
+__device__ __forceinline__ void wait_bar_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) return;
+    }
+}
+
+__device__ __forceinline__ int find_request(const int32_t* row_start, int B, int64_t r) {
+    int lo = 0, hi = B - 1;  // largest b with row_start[b] <= r
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (row_start[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ Seg make_seg(const StreamArgs& a, const int32_t* row_start, int64_t r, int64_t bg,
+                                        int64_t eg) {
+    Seg g;
+    const int64_t rs = r * a.V;
+    g.c0 = max(bg, rs) - rs;
+    g.c1 = min(eg, rs + a.V) - rs;
+    g.b = find_request(row_start, a.B, r);
+    g.k = (int32_t)(r - row_start[g.b]);
+    g.ptr = a.logits + ((int64_t)g.b * a.K + g.k) * a.ld * a.elt;
+    const uint64_t addr0 = reinterpret_cast<uint64_t>(g.ptr) + (uint64_t)(g.c0 * a.elt);
+    const int64_t pad = (int64_t)((16u - (uint32_t)(addr0 & 15u)) & 15u) / a.elt;
+    g.a0 = min(g.c0 + pad, g.c1);
+    g.a1 = g.a0 + (((g.c1 - g.a0) * a.elt) / 16) * 16 / a.elt;
+    const int64_t ce = STAGE_BYTES / a.elt;
+    const int64_t nch = (g.a1 - g.a0 + ce - 1) / ce;
+    g.nchunks = (int32_t)(nch > 0 ? nch : 1);
+    return g;
+}
+
+__device__ __forceinline__ float load_elem(const char* ptr, int64_t i, int elt) {
+    if (elt == 2) {
+        const uint16_t h = __ldg(reinterpret_cast<const unsigned short*>(ptr) + i);
+        return __uint_as_float((uint32_t)h << 16);
+    }
+    return __ldg(reinterpret_cast<const float*>(ptr) + i);
+}
+
+// (m, s) represents sum_i exp(x_i) = exp(m) * s, with s accumulated as
+// sum_i 2^(x_i*log2(e) - m*log2(e)).
+__device__ __forceinline__ void combine(float& m, float& s, float m2, float s2) {
+    const float M = fmaxf(m, m2);
+    const float a = (m == M) ? s : s * ex2_approx((m - M) * L2E);
+    const float b = (m2 == M) ? s2 : s2 * ex2_approx((m2 - M) * L2E);
+    m = M;
+    s = a + b;
+}
+
+__device__ __forceinline__ void warp_combine(float& m, float& s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        combine(m, s, m2, s2);
+    }
+}
+
+__device__ __forceinline__ void lane_add(float& m, float& s, float x) {
+    if (x > m) {
+        s = s * ex2_approx((m - x) * L2E) + 1.0f;
+        m = x;
+    } else if (x != -INFINITY) {
+        s += ex2_approx((x - m) * L2E);  // a NaN lands here and poisons s
+    }
+}
+
+// This lane's share (VPL vectors, lane-interleaved) of one staged chunk.
+template <bool BF16>
+__device__ __forceinline__ void lane_consume(const uint4* stage, int nvec, int vbase, float& m, float& s) {
+    constexpr uint32_t NEG = BF16 ? 0xFF80FF80u : 0xFF800000u;
+    uint4 q[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int idx = vbase + j * (NCW * 32);
+        q[j] = idx < nvec ? stage[idx] : make_uint4(NEG, NEG, NEG, NEG);
+    }
+    float mx;
+    if constexpr (BF16) {
+        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&q[0].x);
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h = __hmax2(h, *reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        }
+        mx = fmaxf(__low2float(h), __high2float(h));
+    } else {
+        mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            mx = fmaxf(mx, fmaxf(fmaxf(__uint_as_float(q[j].x), __uint_as_float(q[j].y)),
+                                 fmaxf(__uint_as_float(q[j].z), __uint_as_float(q[j].w))));
+        }
+    }
+    if (mx > m) {
+        s *= ex2_approx((m - mx) * L2E);
+        m = mx;
+    }
+    const float nmL = (m == -INFINITY) ? 0.f : -m * L2E;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+        if constexpr (BF16) {
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                acc0 += ex2_approx(fmaf(__uint_as_float(w[e] << 16), L2E, nmL));
+                acc1 += ex2_approx(fmaf(__uint_as_float(w[e] & 0xFFFF0000u), L2E, nmL));
+                acc2 += ex2_approx(fmaf(__uint_as_float(w[e + 1] << 16), L2E, nmL));
+                acc3 += ex2_approx(fmaf(__uint_as_float(w[e + 1] & 0xFFFF0000u), L2E, nmL));
+            }
+        } else {
+            acc0 += ex2_approx(fmaf(__uint_as_float(w[0]), L2E, nmL));
+            acc1 += ex2_approx(fmaf(__uint_as_float(w[1]), L2E, nmL));
+            acc2 += ex2_approx(fmaf(__uint_as_float(w[2]), L2E, nmL));
+            acc3 += ex2_approx(fmaf(__uint_as_float(w[3]), L2E, nmL));
+        }
+    }
+    s += (acc0 + acc1) + (acc2 + acc3);
+}
+
+// The row's log-sum-exp is known: write the scores of the trie children of
+// the row's beam.  One warp.
+__device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
+    const int lane = threadIdx.x & 31;
+    const float lse = m + logf(s);
+    if (!isfinite(lse)) {
+        if (lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
+    }
+    const int64_t bk = (int64_t)sg.b * a.K + sg.k;
+    const int t = a.t;
+    const int32_t n = a.node[bk];
+    if (n < 0 || n >= a.trie.nodes[t]) {
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const int32_t lo = a.trie.child_off[t][n], hi = a.trie.child_off[t][n + 1];
+    const int32_t base = a.cand_off[(int64_t)sg.b * (a.K + 1) + sg.k];
+    if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) {
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const float sc = a.score[bk];
+    const int32_t* codes = a.trie.code[t + 1] + lo;
+    const int32_t tb = a.trie.tok_base[t];
+    float* out = a.cand + (int64_t)sg.b * a.cand_stride + base;
+    const int32_t nch = hi - lo;
+    for (int32_t i = lane; i < nch; i += 32) {
+        const float x = load_elem(sg.ptr, tb + codes[i], a.elt);
+        out[i] = sc + (x - lse);
+    }
+}
+
+// Called by the warp that combined this CTA's partial for row r.
+__device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
+                               float s) {
+    const int lane = threadIdx.x & 31;
+    const int64_t fc = (r * a.V) / Q;
+    const int64_t lc = ((r + 1) * a.V - 1) / Q;
+    if (fc == lc) {
+        finish_row(a, sg, m, s);
+        return;
+    }
+    const int side = (r == r_first) ? 0 : 1;
+    int old = 0;
+    if (lane == 0) {
+        a.partial[(int64_t)blockIdx.x * 2 + side] = make_float2(m, s);
+        __threadfence();
+        old = atomicAdd(&a.row_cnt[r], 1);
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != (int)(lc - fc)) return;
+    __threadfence();
+    float M = -INFINITY, S = 0.f;
+    for (int64_t base = fc; base <= lc; base += 32) {
+        const int64_t gg = base + lane;
+        float pm = -INFINITY, ps = 0.f;
+        if (gg <= lc) {
+            const int sd = ((gg * Q) / a.V == r) ? 0 : 1;
+            const float2 p = __ldcg(&a.partial[gg * 2 + sd]);
+            pm = p.x;
+            ps = p.y;
+        }
+        warp_combine(pm, ps);
+        combine(M, S, pm, ps);
+    }
+    if (lane == 0) a.row_cnt[r] = 0;
+    finish_row(a, sg, M, S);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* ring = smem;
+    SmemHdr* hdr = reinterpret_cast<SmemHdr*>(smem + STAGES * STAGE_BYTES);
+    int32_t* row_start = reinterpret_cast<int32_t*>(hdr + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (warp == 0) {  // row_start = exclusive scan of the live counts
+        const int per = (a.B + 31) / 32;
+        int sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int b = lane * per + i;
+            if (b < a.B) sum += min(max(a.live[b], 0), a.K);
+        }
+        const int incl = warp_incl_scan(sum);
+        int run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int b = lane * per + i;
+            if (b < a.B) {
+                row_start[b] = run;
+                run += min(max(a.live[b], 0), a.K);
+            }
+        }
+        if (lane == 31) row_start[a.B] = incl;
+    }
+    if (threadIdx.x == 32) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&hdr->full[i], 1);
+            mbar_init(&hdr->empty[i], NCW);
+            hdr->segcnt[i] = 0;
+        }
+        hdr->abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int64_t E = (int64_t)row_start[a.B] * a.V;
+    if (E == 0) return;
+    const int64_t G = gridDim.x;
+    const int64_t Q = ((E + G - 1) / G + GRAN - 1) / GRAN * GRAN;
+    const int64_t bg = min(E, (int64_t)blockIdx.x * Q);
+    const int64_t eg = min(E, (int64_t)(blockIdx.x + 1) * Q);
+    if (bg >= eg) return;
+    const int64_t r_first = bg / a.V, r_last = (eg - 1) / a.V;
+    const int64_t ce = STAGE_BYTES / a.elt;
+
+    if (warp == NCW) {  // producer
+        if (lane == 0) {
+            uint32_t chunk = 0;
+            bool ok = true;
+            for (int64_t r = r_first; r <= r_last && ok; ++r) {
+                const Seg sg = make_seg(a, row_start, r, bg, eg);
+                for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
+                    const int st = (int)(chunk % STAGES);
+                    const uint32_t ph = (chunk / STAGES) & 1u;
+                    if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const int64_t x0 = sg.a0 + j * ce;
+                    const int64_t x1 = min(sg.a1, x0 + ce);
+                    const uint32_t bytes = (uint32_t)((x1 - x0) * a.elt);
+                    if (bytes) {
+                        mbar_arrive_expect_tx(&hdr->full[st], bytes);
+                        bulk_g2s(ring + (size_t)st * STAGE_BYTES, sg.ptr + x0 * a.elt, bytes, &hdr->full[st]);
+                    } else {
+                        mbar_arrive(&hdr->full[st]);
+                    }
+                }
+            }
+            if (!ok) {
+                const uint32_t first = chunk > (uint32_t)STAGES ? chunk - STAGES : 0u;
+                for (uint32_t c = first; c < chunk; ++c) wait_bar_drain(&hdr->full[c % STAGES], (c / STAGES) & 1u);
+            }
+        }
+        return;
+    }
+
+    // consumers
+    const int cw = warp;
+    uint32_t chunk = 0;
+    float m = -INFINITY, s = 0.f;
+    for (int64_t r = r_first; r <= r_last; ++r) {
+        const Seg sg = make_seg(a, row_start, r, bg, eg);
+        for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
+            const int st = (int)(chunk % STAGES);
+            const uint32_t ph = (chunk / STAGES) & 1u;
+            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err)) return;
+            if (j == 0 && cw == 0 && lane < sg.a0 - sg.c0) lane_add(m, s, load_elem(sg.ptr, sg.c0 + lane, a.elt));
+            const int64_t x0 = sg.a0 + j * ce;
+            const int nvec = (int)(((min(sg.a1, x0 + ce) - x0) * a.elt) / 16);
+            if (nvec > 0)
+                lane_consume<BF16>(reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES), nvec,
+                                   cw * 32 + lane, m, s);
+            const bool last = (j == sg.nchunks - 1);
+            if (last && cw == 0 && lane < sg.c1 - sg.a1) lane_add(m, s, load_elem(sg.ptr, sg.a1 + lane, a.elt));
+            if (!last) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&hdr->empty[st]);
+                continue;
+            }
+            // end of this CTA's segment of row r
+            warp_combine(m, s);
+            if (lane == 0) hdr->part[st][cw] = make_float2(m, s);
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) {
+                __threadfence_block();
+                old = atomicAdd(&hdr->segcnt[st], 1);
+            }
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old == NCW - 1) {
+                __threadfence_block();
+                float pm = -INFINITY, ps = 0.f;
+                if (lane < NCW) {
+                    pm = hdr->part[st][lane].x;
+                    ps = hdr->part[st][lane].y;
+                }
+                warp_combine(pm, ps);
+                __syncwarp();
+                if (lane == 0) {
+                    hdr->segcnt[st] = 0;
+                    mbar_arrive(&hdr->empty[st]);
+                }
+                finish_segment(a, sg, r, r_first, Q, pm, ps);
+            } else {
+                if (lane == 0) mbar_arrive(&hdr->empty[st]);
+            }
+            m = -INFINITY;
+            s = 0.f;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Selection and reorder.
+
+constexpr int SEL_THREADS = 1024;
+constexpr int HBITS = 12;
+constexpr int HBINS = 1 << HBITS;
+static_assert(HBINS == 4 * SEL_THREADS, "each thread owns four histogram bins");
+static_assert(FR_MAX_K <= SEL_THREADS, "one thread per beam slot");
+
+struct SelectArgs {
+    StateDev cur, nxt;
+    TrieDev trie;
+    int32_t B, K, D, t;
+    const float* cand;
+    int64_t cand_stride;
+    int32_t* parent_out;
+    int32_t* token_out;
+    int32_t* err;
+};
+
+__device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t* out_or) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v_and = __reduce_and_sync(0xffffffffu, v_and);
+    v_or = __reduce_or_sync(0xffffffffu, v_or);
+    if (lane == 0) {
+        red[warp] = v_and;
+        red[32 + warp] = v_or;
+    }
+    __syncthreads();
+    const int nw = blockDim.x >> 5;
+    uint32_t a = 0xFFFFFFFFu, o = 0u;
+    for (int w = 0; w < nw; ++w) {
+        a &= red[w];
+        o |= red[32 + w];
+    }
+    __syncthreads();
+    *out_or = o;
+    return a;
+}
+
+// Next step's candidate offsets of request b: exclusive scan over slots of
+// the child counts of each live slot's node.  Called by all threads.
+__device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, const int32_t* node_row, int live,
+                                               int K, int32_t* cand_off_row) {
+    const int j = threadIdx.x;
+    int cnt = 0;
+    if (j < live) {
+        const int32_t n = node_row[j];
+        if (n >= 0) cnt = trie.child_off[t_next][n + 1] - trie.child_off[t_next][n];
+    }
+    int tot;
+    const int e = block_excl_scan(cnt, &tot);
+    if (j < K) cand_off_row[j] = e;
+    if (j == 0) cand_off_row[K] = tot;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
+    __shared__ int32_t s_off[FR_MAX_K + 1];
+    __shared__ int32_t hist[HBINS];
+    __shared__ unsigned long long sel[FR_MAX_K];
+    __shared__ int32_t s_misc[4];
+    __shared__ uint32_t red[64];
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int K = a.K, D = a.D, t = a.t;
+    const int live = min(max(a.cur.live[b], 0), K);
+    for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
+    __syncthreads();
+    int n = s_off[live];
+    if (n < 0 || (int64_t)n > a.cand_stride) {
+        if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
+        n = 0;
+    }
+    const int Kp = min(K, n);
+    const float* cb = a.cand + (int64_t)b * a.cand_stride;
+
+    if (Kp > 0) {
+        uint32_t va = 0xFFFFFFFFu, vo = 0u;
+        for (int i = tid; i < n; i += SEL_THREADS) {
+            const uint32_t k = float_to_key(cb[i]);
+            va &= k;
+            vo |= k;
+        }
+        uint32_t VO;
+        const uint32_t VA = block_and_or(va, vo, red, &VO);
+        const uint32_t diff = VA ^ VO;
+        uint32_t T;
+        int eq_needed, count_eq;
+        if (diff == 0u) {
+            T = VA;
+            eq_needed = Kp;
+            count_eq = n;
+        } else {
+            int lo = 32 - __clz(diff);  // bits >= lo are the same in every key
+            uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
+            int krem = Kp;
+            count_eq = 0;
+            while (lo > 0) {
+                const int width = min(HBITS, lo);
+                const int shift = lo - width;
+                const uint32_t dmask = (1u << width) - 1u;
+                for (int i = tid; i < HBINS; i += SEL_THREADS) hist[i] = 0;
+                __syncthreads();
+                const uint64_t want = (uint64_t)prefix >> lo;
+                for (int i = tid; i < n; i += SEL_THREADS) {
+                    const uint32_t k = float_to_key(cb[i]);
+                    if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
+                }
+                __syncthreads();
+                int h4[4], tsum = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    h4[q] = hist[tid * 4 + q];
+                    tsum += h4[q];
+                }
+                int tot;
+                const int excl = block_excl_scan(tsum, &tot);
+                int cum = tot - excl - tsum;  // keys in the bins above this thread's
+#pragma unroll
+                for (int q = 3; q >= 0; --q) {
+                    if (cum < krem && cum + h4[q] >= krem) {
+                        s_misc[0] = tid * 4 + q;
+                        s_misc[1] = cum;
+                        s_misc[2] = h4[q];
+                    }
+                    cum += h4[q];
+                }
+                __syncthreads();
+                const int d = s_misc[0];
+                krem -= s_misc[1];
+                count_eq = s_misc[2];
+                prefix |= (uint32_t)d << shift;
+                lo = shift;
+                __syncthreads();
+            }
+            T = prefix;
+            eq_needed = krem;
+        }
+        // collect the Kp winners: every key > T and the eq_needed lowest slots with key == T
+        if (tid == 0) s_misc[3] = 0;
+        __syncthreads();
+        if (eq_needed >= count_eq) {
+            for (int i = tid; i < n; i += SEL_THREADS) {
+                const uint32_t k = float_to_key(cb[i]);
+                if (k >= T) {
+                    const int p = atomicAdd(&s_misc[3], 1);
+                    if (p < FR_MAX_K) sel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
+                }
+            }
+        } else {
+            int run_eq = 0;
+            for (int base = 0; base < n; base += SEL_THREADS) {
+                const int i = base + tid;
+                const uint32_t k = i < n ? float_to_key(cb[i]) : 0u;
+                const bool gt = i < n && k > T;
+                const bool eq = i < n && k == T;
+                int tot;
+                const int r = block_excl_scan(eq ? 1 : 0, &tot);
+                if (gt || (eq && run_eq + r < eq_needed)) {
+                    const int p = atomicAdd(&s_misc[3], 1);
+                    if (p < FR_MAX_K) sel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
+                }
+                run_eq += tot;
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && s_misc[3] != Kp) set_error(a.err, FR_ERR_DEVICE);
+        // bitonic sort, descending, over the next power of two
+        int P = 1;
+        while (P < Kp) P <<= 1;
+        for (int i = Kp + tid; i < P; i += SEL_THREADS) sel[i] = 0ull;
+        __syncthreads();
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int i = tid; i < P; i += SEL_THREADS) {
+                    const int ixj = i ^ j;
+                    if (ixj > i) {
+                        const unsigned long long x = sel[i], y = sel[ixj];
+                        const bool swap = ((i & k) == 0) ? (x < y) : (x > y);
+                        if (swap) {
+                            sel[i] = y;
+                            sel[ixj] = x;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+    }
+
+    // emit survivors (thread j = slot j)
+    const int j = tid;
+    int32_t child = -1;
+    if (j < K) {
+        const int64_t oj = (int64_t)b * K + j;
+        if (j < Kp) {
+            const unsigned long long v = sel[j];
+            const uint32_t key = (uint32_t)(v >> 32);
+            const int32_t slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
+            int lo = 0, hi = live - 1;  // parent: last k with s_off[k] <= slot
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
+            }
+            const int k = lo;
+            const int64_t ok = (int64_t)b * K + k;
+            const int32_t np = a.cur.node[ok];
+            int32_t tok = -1;
+            if (np >= 0 && np < a.trie.nodes[t]) {
+                child = a.trie.child_off[t][np] + (slot - s_off[k]);
+                if (child >= 0 && child < a.trie.nodes[t + 1]) {
+                    tok = a.trie.tok_base[t] + a.trie.code[t + 1][child];
+                } else {
+                    child = -1;
+                }
+            }
+            if (child < 0) set_error(a.err, FR_ERR_DEVICE);
+            a.nxt.node[oj] = child;
+            a.nxt.score[oj] = key_to_float(key);
+            a.nxt.kv[oj] = a.cur.kv[ok];
+            a.parent_out[oj] = k;
+            a.token_out[oj] = tok;
+            for (int l = 0; l < D; ++l)
+                a.nxt.prefix[oj * D + l] = (l < t) ? a.cur.prefix[ok * D + l] : (l == t ? tok : -1);
+        } else {
+            a.nxt.node[oj] = -1;
+            a.nxt.score[oj] = -INFINITY;
+            a.nxt.kv[oj] = -1;
+            a.parent_out[oj] = -1;
+            a.token_out[oj] = -1;
+            for (int l = 0; l < D; ++l) a.nxt.prefix[oj * D + l] = -1;
+        }
+    }
+    if (tid == 0) a.nxt.live[b] = Kp;
+    if (t + 1 < D) {
+        // node ids of the survivors are in registers of threads 0..Kp-1
+        const int jj = threadIdx.x;
+        int cnt = 0;
+        if (jj < Kp && child >= 0) cnt = a.trie.child_off[t + 1][child + 1] - a.trie.child_off[t + 1][child];
+        int tot;
+        const int e = block_excl_scan(cnt, &tot);
+        int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
+        if (jj < K) row[jj] = e;
+        if (jj == 0) row[K] = tot;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// State kernels.
+
+__global__ void k_reset(StateDev s0, int32_t B, int32_t K, int32_t D, TrieDev trie) {
+    const int64_t nbk = (int64_t)B * K;
+    const int32_t root_fan = trie.child_off[0][1] - trie.child_off[0][0];
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t b = (int32_t)(i / K), k = (int32_t)(i % K);
+        const bool root = (k == 0);
+        s0.node[i] = root ? 0 : -1;
+        s0.score[i] = root ? 0.f : -INFINITY;
+        s0.kv[i] = root ? b * K : -1;
+        for (int l = 0; l < D; ++l) s0.prefix[i * D + l] = -1;
+        if (root) s0.live[b] = 1;
+    }
+    const int64_t no = (int64_t)B * (K + 1);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < no; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t j = (int32_t)(i % (K + 1));
+        s0.cand_off[i] = (j == 0) ? 0 : root_fan;
+    }
+}
+
+// Locates every live prefix (codes) in the trie; writes node ids and tokens.
+__global__ void k_walk(StateDev st, int32_t B, int32_t K, int32_t D, int32_t t, TrieDev trie,
+                       const int32_t* __restrict__ codes, const int32_t* __restrict__ kv_given, int32_t* err) {
+    const int64_t nbk = (int64_t)B * K;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t b = (int32_t)(i / K), k = (int32_t)(i % K);
+        const int32_t live = min(max(st.live[b], 0), K);
+        if (k < live) {
+            int32_t node = 0;
+            for (int l = 0; l < t && node >= 0; ++l) {
+                const int32_t c = codes[i * D + l];
+                int32_t lo = trie.child_off[l][node], hi = trie.child_off[l][node + 1];
+                const int32_t* cl = trie.code[l + 1];
+                while (lo < hi) {  // first child with code >= c
+                    const int32_t mid = (lo + hi) >> 1;
+                    if (cl[mid] < c) lo = mid + 1; else hi = mid;
+                }
+                if (lo < trie.child_off[l][node + 1] && cl[lo] == c) {
+                    node = lo;
+                    st.prefix[i * D + l] = trie.tok_base[l] + c;
+                } else {
+                    node = -1;
+                }
+            }
+            if (node < 0) set_error(err, FR_ERR_NOT_IN_CATALOG);
+            for (int l = t; l < D; ++l) st.prefix[i * D + l] = -1;
+            st.node[i] = node;
+            st.kv[i] = kv_given ? kv_given[i] : b * K + k;
+        } else {
+            st.node[i] = -1;
+            st.score[i] = -INFINITY;
+            st.kv[i] = -1;
+            for (int l = 0; l < D; ++l) st.prefix[i * D + l] = -1;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) k_cand_off(StateDev st, int32_t K, int32_t t, TrieDev trie) {
+    const int b = blockIdx.x;
+    const int live = min(max(st.live[b], 0), K);
+    write_cand_off(trie, t, st.node + (int64_t)b * K, live, K, st.cand_off + (int64_t)b * (K + 1));
+}
+
+__global__ void k_finalize(StateDev st, int32_t B, int32_t K, int32_t D, TrieDev trie, int32_t* __restrict__ sids,
+                           float* __restrict__ scores, int32_t* __restrict__ items) {
+    const int64_t nbk = (int64_t)B * K;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t node = st.node[i];
+        if (node >= 0) {
+            for (int l = 0; l < D; ++l) sids[i * D + l] = st.prefix[i * D + l] - trie.tok_base[l];
+            scores[i] = st.score[i];
+            if (items) items[i] = trie.leaf_row[node];
+        } else {
+            for (int l = 0; l < D; ++l) sids[i * D + l] = -1;
+            scores[i] = -INFINITY;
+            if (items) items[i] = -1;
+        }
+    }
+}
+
+int small_grid(int64_t n) {
+    const int64_t g = (n + 255) / 256;
+    return (int)(g < 1 ? 1 : (g > 4096 ? 4096 : g));
+}
+
+}  // namespace
+
+size_t stream_smem_bytes(int32_t B) {
+    return (size_t)STAGES * STAGE_BYTES + sizeof(SmemHdr) + sizeof(int32_t) * (size_t)(B + 1);
+}
+
+cudaError_t stream_kernel_setup() {
+    const int max_bytes = (int)stream_smem_bytes(FR_MAX_B);
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+}
+
+cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, const void* logits,
+                          int64_t ld, cudaStream_t s) {
+    const StateDev& cur = buf.st[t & 1];
+    StreamArgs a;
+    a.logits = static_cast<const char*>(logits);
+    a.ld = ld;
+    a.V = sh.V;
+    a.B = sh.B;
+    a.K = sh.K;
+    a.t = t;
+    a.elt = sh.dtype == FR_BF16 ? 2 : 4;
+    a.live = cur.live;
+    a.node = cur.node;
+    a.score = cur.score;
+    a.cand_off = cur.cand_off;
+    a.trie = trie;
+    a.cand = buf.cand;
+    a.cand_stride = buf.cand_stride;
+    a.partial = buf.partial;
+    a.row_cnt = buf.row_cnt;
+    a.err = buf.err;
+    const size_t smem = stream_smem_bytes(sh.B);
+    if (sh.dtype == FR_BF16)
+        k_stream<true><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
+    else
+        k_stream<false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, cudaStream_t s) {
+    SelectArgs a;
+    a.cur = buf.st[t & 1];
+    a.nxt = buf.st[(t + 1) & 1];
+    a.trie = trie;
+    a.B = sh.B;
+    a.K = sh.K;
+    a.D = sh.D;
+    a.t = t;
+    a.cand = buf.cand;
+    a.cand_stride = buf.cand_stride;
+    a.parent_out = buf.parent;
+    a.token_out = buf.token;
+    a.err = buf.err;
+    k_select<<<sh.B, SEL_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s) {
+    const int64_t nbk = (int64_t)sh.B * sh.K;
+    k_reset<<<small_grid(nbk + sh.B), 256, 0, s>>>(buf.st[0], sh.B, sh.K, sh.D, trie);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(buf.parent, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(buf.token, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(buf.row_cnt, 0, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
+    return cudaMemsetAsync(buf.err, 0, sizeof(int32_t), s);
+}
+
+cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
+                             const int32_t* prefix_codes, const int32_t* kv_given, cudaStream_t s) {
+    const StateDev& st = buf.st[t & 1];
+    const int64_t nbk = (int64_t)sh.B * sh.K;
+    k_walk<<<small_grid(nbk), 256, 0, s>>>(st, sh.B, sh.K, sh.D, t, trie, prefix_codes, kv_given, buf.err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (t < sh.D) {
+        k_cand_off<<<sh.B, SEL_THREADS, 0, s>>>(st, sh.K, t, trie);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if ((e = cudaMemsetAsync(buf.parent, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(buf.token, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
+    return cudaMemsetAsync(buf.row_cnt, 0, sizeof(int32_t) * (size_t)nbk, s);
+}
+
+cudaError_t launch_finalize(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, int32_t* sids,
+                            float* scores, int32_t* items, cudaStream_t s) {
+    const int64_t nbk = (int64_t)sh.B * sh.K;
+    k_finalize<<<small_grid(nbk), 256, 0, s>>>(buf.st[t & 1], sh.B, sh.K, sh.D, trie, sids, scores, items);
+    return cudaGetLastError();
+}
+
+}  // namespace fr

@@ -1,0 +1,41 @@
+// fr_step.cuh -- kernel launchers of the beam step (internal to libfr).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fr_internal.cuh"
+
+namespace fr {
+
+struct StepBuffers {
+    StateDev st[2];
+    int32_t* parent;      // [B*K] latest step
+    int32_t* token;       // [B*K]
+    float* cand;          // [B * cand_stride]
+    int64_t cand_stride;  // K * max_fanout
+    float2* partial;      // [grid * 2] (max, scaled sum) per CTA and row side
+    int32_t* row_cnt;     // [B*K] arrival counters of shared rows
+    int32_t* err;         // sticky device status word
+};
+
+struct StepShape {
+    int32_t B, K, V, D;
+    int32_t dtype;  // fr_dtype
+    int32_t grid;   // CTAs of the streaming kernel
+};
+
+// Streaming kernel: dynamic shared memory it needs for B requests.
+size_t stream_smem_bytes(int32_t B);
+cudaError_t stream_kernel_setup();  // raises the kernel's shared-memory limit
+
+cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
+                          const void* logits, int64_t ld, cudaStream_t s);
+cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, cudaStream_t s);
+cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s);
+cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
+                             const int32_t* prefix_codes, const int32_t* kv_given, cudaStream_t s);
+cudaError_t launch_finalize(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, int32_t* sids,
+                            float* scores, int32_t* items, cudaStream_t s);
+
+}  // namespace fr
