@@ -217,3 +217,47 @@ def test_kv_slots_follow_parents():
             np.testing.assert_array_equal(v.kv[b, :n], prev_kv[b, v.parent[b, :n]])
             assert np.all(v.kv[b, n:] == -1)
         prev_kv = v.kv
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_extreme_logit_ranges(dtype):
+    """Rows whose maximum comes late, jumps far above the first values, or
+    follows a run of -inf: the streaming log-sum-exp moves its reference point
+    (and re-sums a chunk when a term could overflow).  Expected scores are
+    x[token] - logsumexp(row) in double (scipy), on the same rounded values."""
+    import torch
+    from scipy.special import logsumexp
+
+    V, C = 40000, 64
+    w = W("extreme", B=4, K=16, depth=1, C=C, V=V, sid_base=30000, n_items=C, dtype=dtype)
+    sids = np.arange(C, dtype=np.int32).reshape(-1, 1)
+    gpu = GpuBeam(w, sids)
+    try:
+        v = np.arange(V, dtype=np.float64)
+        rows = np.stack([
+            -150.0 + 300.0 * v / V,                                  # rising ramp, max at the end
+            150.0 - 300.0 * v / V,                                   # falling ramp
+            np.where(v == 35000, 100.0, -50.0 + (v % 7) * 0.25),      # late spike far above the rest
+            np.where(v < 20000, -np.inf, np.sin(v) * 3.0),           # long run of -inf first
+        ])
+        t = torch.tensor(rows, dtype=torch.float32)
+        t = t.to(torch.bfloat16) if dtype == "bf16" else t
+        gpu.logits.zero_()
+        gpu.logits[:, 0, :] = t.cuda()
+        fr_rows = t.float().numpy().astype(np.float64)
+        from trie_constrained_beam_fr_b200 import fr
+        fr.fr_beam_reset(gpu.beam)
+        fr.fr_beam_step(gpu.beam, gpu.logits)
+        torch.cuda.synchronize()
+        assert fr.fr_beam_status(gpu.beam) == fr.FR_OK
+        out = gpu.view()
+    finally:
+        gpu.close()
+    for b in range(4):
+        lse = float(logsumexp(fr_rows[b]))
+        lp = fr_rows[b, w.sid_base: w.sid_base + C] - lse
+        order = sorted(range(C), key=lambda c: (-lp[c], c))[: w.K]
+        np.testing.assert_allclose(out.score[b], lp[order], atol=1e-4, rtol=0)
+        gaps = np.abs(np.diff(lp[order]))
+        if np.all(gaps > 1e-4):
+            np.testing.assert_array_equal(out.token[b], w.sid_base + np.array(order))

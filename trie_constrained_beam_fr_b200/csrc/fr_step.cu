@@ -40,23 +40,53 @@
 namespace fr {
 namespace {
 
-constexpr int NCW = 16;  // consumer warps
-constexpr int STREAM_THREADS = (NCW + 1) * 32;
-constexpr int STAGES = 6;
-constexpr int STAGE_BYTES = 32768;
+#ifndef FR_NCW
+#define FR_NCW 16
+#endif
+#ifndef FR_STAGES
+#define FR_STAGES 6
+#endif
+#ifndef FR_STAGE_BYTES
+#define FR_STAGE_BYTES 32768
+#endif
+constexpr int NCW = FR_NCW;  // consumer warps: reduce the staged chunks
+constexpr int NFW = 2;       // finisher warps: lse, cross-CTA combine, candidate scores
+constexpr int PRODUCER_WARP = NCW;
+constexpr int FIRST_FINISHER_WARP = NCW + 1;
+constexpr int STREAM_THREADS = (NCW + 1 + NFW) * 32;
+constexpr int STAGES = FR_STAGES;
+constexpr int STAGE_BYTES = FR_STAGE_BYTES;
+constexpr int RING_BYTES = STAGES * STAGE_BYTES;
 constexpr int VEC_PER_STAGE = STAGE_BYTES / 16;
 constexpr int VPL = VEC_PER_STAGE / (NCW * 32);  // 16-byte vectors per lane per chunk
-constexpr int64_t GRAN = 1024;                   // CTA ranges start at multiples of this many elements
+constexpr int QCAP = 32;    // finished-segment jobs in flight per CTA
+constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
+static_assert(PSLOTS > 2 * STAGES, "partial slots must outnumber the segments in flight");
+constexpr int64_t GRAN = 1024;  // CTA ranges start at multiples of this many elements
 constexpr float L2E = 1.4426950408889634f;
+#ifndef FR_POLY_PAIRS
+#define FR_POLY_PAIRS 0
+#endif
+// Of the four bf16 pairs in each 16-byte vector, this many take exp2 on the
+// FMA pipe (polynomial) instead of the MUFU.
+constexpr int POLY_PAIRS = FR_POLY_PAIRS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
 
+struct Job {
+    int64_t r;  // row whose segment in this CTA is reduced
+    float m, s;
+};
+
 struct SmemHdr {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    float2 part[STAGES][NCW];
-    int32_t segcnt[STAGES];
+    float2 part[PSLOTS][NCW];  // per-warp partials of a segment, slot = segment % PSLOTS
+    int32_t segcnt[PSLOTS];
+    Job jobs[QCAP];
+    int32_t ready[QCAP];  // job id + 1 once jobs[slot] holds that job
+    int32_t freed[QCAP];  // job id + 1 once a finisher has copied it out
     int32_t abort_flag;
     int32_t pad;
 };
@@ -109,6 +139,24 @@ __device__ __forceinline__ void wait_bar_drain(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// Bounded wait until *word == want (a sequence number written by another warp
+// of this CTA).  Returns false on abort or after the time limit.
+__device__ __forceinline__ bool wait_seq(volatile int32_t* word, int32_t want, volatile int32_t* abort_flag,
+                                         int32_t* err) {
+    if (*word == want) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (*word == want) return true;
+        if (*abort_flag) return false;
+        __nanosleep(64);
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            set_error(err, FR_ERR_DEVICE);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ int find_request(const int32_t* row_start, int B, int64_t r) {
     int lo = 0, hi = B - 1;  // largest b with row_start[b] <= r
     while (lo < hi) {
@@ -118,21 +166,23 @@ __device__ __forceinline__ int find_request(const int32_t* row_start, int B, int
     return lo;
 }
 
+template <int ELT>
 __device__ __forceinline__ Seg make_seg(const StreamArgs& a, const int32_t* row_start, int64_t r, int64_t bg,
                                         int64_t eg) {
+    constexpr int64_t VE = 16 / ELT;          // elements per 16-byte vector
+    constexpr int64_t CE = STAGE_BYTES / ELT;  // elements per chunk
     Seg g;
     const int64_t rs = r * a.V;
     g.c0 = max(bg, rs) - rs;
     g.c1 = min(eg, rs + a.V) - rs;
     g.b = find_request(row_start, a.B, r);
     g.k = (int32_t)(r - row_start[g.b]);
-    g.ptr = a.logits + ((int64_t)g.b * a.K + g.k) * a.ld * a.elt;
-    const uint64_t addr0 = reinterpret_cast<uint64_t>(g.ptr) + (uint64_t)(g.c0 * a.elt);
-    const int64_t pad = (int64_t)((16u - (uint32_t)(addr0 & 15u)) & 15u) / a.elt;
+    g.ptr = a.logits + ((int64_t)g.b * a.K + g.k) * a.ld * ELT;
+    const uint32_t mis = (uint32_t)(reinterpret_cast<uint64_t>(g.ptr) + (uint64_t)(g.c0 * ELT)) & 15u;
+    const int64_t pad = (int64_t)((16u - mis) & 15u) / ELT;
     g.a0 = min(g.c0 + pad, g.c1);
-    g.a1 = g.a0 + (((g.c1 - g.a0) * a.elt) / 16) * 16 / a.elt;
-    const int64_t ce = STAGE_BYTES / a.elt;
-    const int64_t nch = (g.a1 - g.a0 + ce - 1) / ce;
+    g.a1 = g.a0 + ((g.c1 - g.a0) & ~(VE - 1));
+    const int64_t nch = (g.a1 - g.a0 + CE - 1) / CE;
     g.nchunks = (int32_t)(nch > 0 ? nch : 1);
     return g;
 }
@@ -164,68 +214,180 @@ __device__ __forceinline__ void warp_combine(float& m, float& s) {
     }
 }
 
-__device__ __forceinline__ void lane_add(float& m, float& s, float x) {
-    if (x > m) {
-        s = s * ex2_approx((m - x) * L2E) + 1.0f;
-        m = x;
-    } else if (x != -INFINITY) {
-        s += ex2_approx((x - m) * L2E);  // a NaN lands here and poisons s
-    }
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes
+// of data).
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 ex2_pair(f32x2 v) {
+    float lo, hi;
+    unpack2(v, lo, hi);
+    return pack2(ex2_approx(lo), ex2_approx(hi));
 }
 
-// This lane's share (VPL vectors, lane-interleaved) of one staged chunk.
-template <bool BF16>
-__device__ __forceinline__ void lane_consume(const uint4* stage, int nvec, int vbase, float& m, float& s) {
-    constexpr uint32_t NEG = BF16 ? 0xFF80FF80u : 0xFF800000u;
-    uint4 q[VPL];
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        const int idx = vbase + j * (NCW * 32);
-        q[j] = idx < nvec ? stage[idx] : make_uint4(NEG, NEG, NEG, NEG);
-    }
-    float mx;
-    if constexpr (BF16) {
-        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&q[0].x);
-#pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) h = __hmax2(h, *reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-        }
-        mx = fmaxf(__low2float(h), __high2float(h));
-    } else {
-        mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            mx = fmaxf(mx, fmaxf(fmaxf(__uint_as_float(q[j].x), __uint_as_float(q[j].y)),
-                                 fmaxf(__uint_as_float(q[j].z), __uint_as_float(q[j].w))));
-        }
-    }
-    if (mx > m) {
-        s *= ex2_approx((m - mx) * L2E);
-        m = mx;
-    }
-    const float nmL = (m == -INFINITY) ? 0.f : -m * L2E;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+// 2^y for a pair on the FMA pipe instead of the MUFU: Cody-Waite reduction
+// y = n + f, n = round(y), f in [-1/2, 1/2], then a degree-5 minimax
+// polynomial for 2^f (relative error 1.5e-7 after rounding the coefficients
+// to float32; coefficients from gen_exp2_poly.py, a Remez fit), then n is
+// added to the exponent field.  Valid for finite y <= 126; y is clamped below
+// at -125, where 2^y is negligible next to any sum it joins.
+__device__ __forceinline__ f32x2 exp2_poly_pair(f32x2 y) {
+    constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+    float y0, y1;
+    unpack2(y, y0, y1);
+    const f32x2 yc = pack2(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
+    const f32x2 t = add2(yc, pack2(MAGIC, MAGIC));       // low mantissa bits hold n
+    const f32x2 f = sub2(yc, sub2(t, pack2(MAGIC, MAGIC)));  // exact
+    f32x2 p = fma2(pack2(1.327647245e-03f, 1.327647245e-03f), f, pack2(9.675540961e-03f, 9.675540961e-03f));
+    p = fma2(p, f, pack2(5.550713092e-02f, 5.550713092e-02f));
+    p = fma2(p, f, pack2(2.402212024e-01f, 2.402212024e-01f));
+    p = fma2(p, f, pack2(6.931469440e-01f, 6.931469440e-01f));
+    p = fma2(p, f, pack2(1.000000119e+00f, 1.000000119e+00f));
+    float p0, p1, t0, t1;
+    unpack2(p, p0, p1);
+    unpack2(t, t0, t1);
+    // bits(t) = bits(MAGIC) + n and bits(MAGIC) << 23 == 0 (mod 2^32), so
+    // bits(t) << 23 == n << 23: the exponent increment.
+    return pack2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// Exponent sum of this lane's VPL vectors against the reference point mref:
+// sum 2^(x*log2(e) - mref*log2(e)), in packed pairs.
+template <bool BF16, int POLY>
+__device__ __forceinline__ f32x2 lane_expsum(const uint4 (&q)[VPL], float mref) {
+    const float nmL = (mref == -INFINITY) ? 0.f : -mref * L2E;
+    const f32x2 c2 = pack2(nmL, nmL);
+    const f32x2 l2 = pack2(L2E, L2E);
+    f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
         const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
         if constexpr (BF16) {
 #pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-                acc0 += ex2_approx(fmaf(__uint_as_float(w[e] << 16), L2E, nmL));
-                acc1 += ex2_approx(fmaf(__uint_as_float(w[e] & 0xFFFF0000u), L2E, nmL));
-                acc2 += ex2_approx(fmaf(__uint_as_float(w[e + 1] << 16), L2E, nmL));
-                acc3 += ex2_approx(fmaf(__uint_as_float(w[e + 1] & 0xFFFF0000u), L2E, nmL));
+            for (int e = 0; e < 4; ++e) {
+                const f32x2 x = pack2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+                const f32x2 y = fma2(x, l2, c2);
+                acc[e] = add2(acc[e], (e < POLY) ? exp2_poly_pair(y) : ex2_pair(y));
             }
         } else {
-            acc0 += ex2_approx(fmaf(__uint_as_float(w[0]), L2E, nmL));
-            acc1 += ex2_approx(fmaf(__uint_as_float(w[1]), L2E, nmL));
-            acc2 += ex2_approx(fmaf(__uint_as_float(w[2]), L2E, nmL));
-            acc3 += ex2_approx(fmaf(__uint_as_float(w[3]), L2E, nmL));
+            const f32x2 x0 = pack2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+            const f32x2 x1 = pack2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+            acc[(2 * j) & 3] = add2(acc[(2 * j) & 3], ex2_pair(fma2(x0, l2, c2)));
+            acc[(2 * j + 1) & 3] = add2(acc[(2 * j + 1) & 3], ex2_pair(fma2(x1, l2, c2)));
         }
     }
-    s += (acc0 + acc1) + (acc2 + acc3);
+    return add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+}
+
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// Largest value of this lane's VPL vectors; NaN if any value is NaN.
+template <bool BF16>
+__device__ __forceinline__ float lane_max(const uint4 (&q)[VPL]) {
+    if constexpr (BF16) {
+        __nv_bfloat162 h[4];
+        {
+            const uint32_t w0[4] = {q[0].x, q[0].y, q[0].z, q[0].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = *reinterpret_cast<const __nv_bfloat162*>(&w0[e]);
+        }
+#pragma unroll
+        for (int j = 1; j < VPL; ++j) {
+            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = __hmax2_nan(h[e], *reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        }
+        const __nv_bfloat162 hm = __hmax2_nan(__hmax2_nan(h[0], h[1]), __hmax2_nan(h[2], h[3]));
+        return fmax_nan(__low2float(hm), __high2float(hm));
+    } else {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            m4[0] = fmax_nan(m4[0], __uint_as_float(q[j].x));
+            m4[1] = fmax_nan(m4[1], __uint_as_float(q[j].y));
+            m4[2] = fmax_nan(m4[2], __uint_as_float(q[j].z));
+            m4[3] = fmax_nan(m4[3], __uint_as_float(q[j].w));
+        }
+        return fmax_nan(fmax_nan(m4[0], m4[1]), fmax_nan(m4[2], m4[3]));
+    }
+}
+
+// This lane's share (VPL 16-byte vectors, lane-interleaved) of one staged
+// chunk (already in registers; lanes past the chunk's end hold -inf), folded
+// into its running (reference m, packed scaled sum s2), where
+// sum exp(x) = exp(m) * (s2.lo + s2.hi).  The exponents are taken against
+// the reference the lane already holds (or its first element), so they do not
+// wait for the chunk's maximum; the maximum, computed alongside, moves the
+// reference afterwards when it rose by more than 16 (nats), and in the rare
+// case that it rose by more than 80 -- where a term could overflow -- the
+// chunk is summed again against the new maximum.
+template <bool BF16>
+__device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f32x2& s2) {
+    float mref = m;
+    if (mref == -INFINITY) mref = BF16 ? __uint_as_float(q[0].x << 16) : __uint_as_float(q[0].x);
+    f32x2 part = lane_expsum<BF16, BF16 ? POLY_PAIRS : 0>(q, mref);
+    const float mx = lane_max<BF16>(q);
+    if (!(mref > -INFINITY && mx <= mref + 80.f)) {
+        // reference unusable (-inf/NaN first element), a term may overflow,
+        // or the chunk holds a NaN / +inf: sum again on the MUFU alone, which
+        // keeps NaN and infinities intact
+        mref = fmaxf(mx, mref);
+        if (m != -INFINITY) {
+            const float sc = ex2_approx((m - mref) * L2E);
+            s2 = mul2(s2, pack2(sc, sc));
+        }
+        part = lane_expsum<BF16, 0>(q, mref);
+    }
+    s2 = add2(s2, part);
+    m = mref;
+    if (mx > m + 16.f) {
+        const float sc = ex2_approx((m - mx) * L2E);
+        s2 = mul2(s2, pack2(sc, sc));
+        m = mx;
+    }
+}
+
+// One element (ragged head / tail of a segment) into (m, s2).
+__device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
+    if (x > m) {
+        const float sc = ex2_approx((m - x) * L2E);
+        s2 = add2(mul2(s2, pack2(sc, sc)), pack2(1.0f, 0.0f));
+        m = x;
+    } else if (x != -INFINITY) {
+        s2 = add2(s2, pack2(ex2_approx((x - m) * L2E), 0.0f));  // a NaN lands here and poisons s
+    }
 }
 
 // The row's log-sum-exp is known: write the scores of the trie children of
@@ -254,9 +416,22 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
     const int32_t tb = a.trie.tok_base[t];
     float* out = a.cand + (int64_t)sg.b * a.cand_stride + base;
     const int32_t nch = hi - lo;
-    for (int32_t i = lane; i < nch; i += 32) {
-        const float x = load_elem(sg.ptr, tb + codes[i], a.elt);
-        out[i] = sc + (x - lse);
+    constexpr int U = 8;  // independent gathers in flight per lane
+    for (int32_t i0 = 0; i0 < nch; i0 += 32 * U) {
+        int32_t code[U];
+        float x[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int32_t i = i0 + u * 32 + lane;
+            code[u] = i < nch ? __ldg(codes + i) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.ptr, tb + code[u], a.elt) : 0.f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int32_t i = i0 + u * 32 + lane;
+            if (i < nch) out[i] = sc + (x[u] - lse);
+        }
     }
 }
 
@@ -299,9 +474,10 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
 
 template <bool BF16>
 __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a) {
+    constexpr int ELT = BF16 ? 2 : 4;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* ring = smem;
-    SmemHdr* hdr = reinterpret_cast<SmemHdr*>(smem + STAGES * STAGE_BYTES);
+    SmemHdr* hdr = reinterpret_cast<SmemHdr*>(smem + RING_BYTES);
     int32_t* row_start = reinterpret_cast<int32_t*>(hdr + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -323,14 +499,20 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
         }
         if (lane == 31) row_start[a.B] = incl;
     }
-    if (threadIdx.x == 32) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&hdr->full[i], 1);
-            mbar_init(&hdr->empty[i], NCW);
-            hdr->segcnt[i] = 0;
+    if (warp == 1) {
+        for (int i = lane; i < QCAP; i += 32) {
+            hdr->ready[i] = 0;
+            hdr->freed[i] = 0;
         }
-        hdr->abort_flag = 0;
-        fence_mbar_init();
+        for (int i = lane; i < PSLOTS; i += 32) hdr->segcnt[i] = 0;
+        if (lane == 0) {
+            for (int i = 0; i < STAGES; ++i) {
+                mbar_init(&hdr->full[i], 1);
+                mbar_init(&hdr->empty[i], NCW);
+            }
+            hdr->abort_flag = 0;
+            fence_mbar_init();
+        }
     }
     __syncthreads();
 
@@ -342,29 +524,35 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
     const int64_t eg = min(E, (int64_t)(blockIdx.x + 1) * Q);
     if (bg >= eg) return;
     const int64_t r_first = bg / a.V, r_last = (eg - 1) / a.V;
-    const int64_t ce = STAGE_BYTES / a.elt;
 
-    if (warp == NCW) {  // producer
+    if (warp == PRODUCER_WARP) {
         if (lane == 0) {
             uint32_t chunk = 0;
+            int st = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int64_t r = r_first; r <= r_last && ok; ++r) {
-                const Seg sg = make_seg(a, row_start, r, bg, eg);
+                const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
+                const char* src = sg.ptr + sg.a0 * ELT;
+                int64_t left = (sg.a1 - sg.a0) * ELT;
                 for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
-                    const int st = (int)(chunk % STAGES);
-                    const uint32_t ph = (chunk / STAGES) & 1u;
                     if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err)) {
                         ok = false;
                         break;
                     }
-                    const int64_t x0 = sg.a0 + j * ce;
-                    const int64_t x1 = min(sg.a1, x0 + ce);
-                    const uint32_t bytes = (uint32_t)((x1 - x0) * a.elt);
+                    const uint32_t bytes =
+                        (uint32_t)(left < (int64_t)STAGE_BYTES ? (left > 0 ? left : 0) : STAGE_BYTES);
                     if (bytes) {
                         mbar_arrive_expect_tx(&hdr->full[st], bytes);
-                        bulk_g2s(ring + (size_t)st * STAGE_BYTES, sg.ptr + x0 * a.elt, bytes, &hdr->full[st]);
+                        bulk_g2s(ring + (size_t)st * STAGE_BYTES, src, bytes, &hdr->full[st]);
                     } else {
                         mbar_arrive(&hdr->full[st]);
+                    }
+                    src += STAGE_BYTES;
+                    left -= STAGE_BYTES;
+                    if (++st == STAGES) {
+                        st = 0;
+                        ph ^= 1u;
                     }
                 }
             }
@@ -376,58 +564,105 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
         return;
     }
 
-    // consumers
-    const int cw = warp;
-    uint32_t chunk = 0;
-    float m = -INFINITY, s = 0.f;
-    for (int64_t r = r_first; r <= r_last; ++r) {
-        const Seg sg = make_seg(a, row_start, r, bg, eg);
-        for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
-            const int st = (int)(chunk % STAGES);
-            const uint32_t ph = (chunk / STAGES) & 1u;
-            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err)) return;
-            if (j == 0 && cw == 0 && lane < sg.a0 - sg.c0) lane_add(m, s, load_elem(sg.ptr, sg.c0 + lane, a.elt));
-            const int64_t x0 = sg.a0 + j * ce;
-            const int nvec = (int)(((min(sg.a1, x0 + ce) - x0) * a.elt) / 16);
-            if (nvec > 0)
-                lane_consume<BF16>(reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES), nvec,
-                                   cw * 32 + lane, m, s);
-            const bool last = (j == sg.nchunks - 1);
-            if (last && cw == 0 && lane < sg.c1 - sg.a1) lane_add(m, s, load_elem(sg.ptr, sg.a1 + lane, a.elt));
-            if (!last) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&hdr->empty[st]);
-                continue;
+    if (warp >= FIRST_FINISHER_WARP) {
+        // Finishers take the reduced segments in order (job j = row r_first + j)
+        // from the queue the consumers fill, so that the gathers of the
+        // candidate scores never hold up the ring.
+        const int64_t njobs = r_last - r_first + 1;
+        for (int64_t j = warp - FIRST_FINISHER_WARP; j < njobs; j += NFW) {
+            const int slot = (int)(j % QCAP);
+            if (!wait_seq(&hdr->ready[slot], (int32_t)(j + 1), &hdr->abort_flag, a.err)) return;
+            __threadfence_block();
+            const Job job = hdr->jobs[slot];
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(j + 1);
             }
-            // end of this CTA's segment of row r
-            warp_combine(m, s);
-            if (lane == 0) hdr->part[st][cw] = make_float2(m, s);
+            const Seg sg = make_seg<ELT>(a, row_start, job.r, bg, eg);
+            finish_segment(a, sg, job.r, r_first, Q, job.m, job.s);
+        }
+        return;
+    }
+
+    // consumers: every warp reduces its lane-interleaved share of each chunk
+    const int cw = warp;
+    const int vbase = cw * 32 + lane;
+    int st = 0;
+    uint32_t ph = 0;
+    float m = -INFINITY;
+    f32x2 s2 = pack2(0.f, 0.f);
+    for (int64_t r = r_first; r <= r_last; ++r) {
+        const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
+        const int32_t nvec_all = (int32_t)((sg.a1 - sg.a0) * ELT / 16);
+        for (int j = 0; j < sg.nchunks; ++j) {
+            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err)) return;
+            if (j == 0 && cw == 0 && lane < sg.a0 - sg.c0) lane_add(m, s2, load_elem(sg.ptr, sg.c0 + lane, ELT));
+            const uint4* stage = reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES);
+            const int32_t nvec = min(nvec_all - j * VEC_PER_STAGE, VEC_PER_STAGE);
+            uint4 q[VPL];
+            if (nvec == VEC_PER_STAGE) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) q[v] = stage[vbase + v * (NCW * 32)];
+                lane_consume<BF16>(q, m, s2);
+            } else if (nvec > 0) {
+                constexpr uint32_t NEG = BF16 ? 0xFF80FF80u : 0xFF800000u;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    const int idx = vbase + v * (NCW * 32);
+                    q[v] = idx < nvec ? stage[idx] : make_uint4(NEG, NEG, NEG, NEG);
+                }
+                lane_consume<BF16>(q, m, s2);
+            }
+            const bool last = (j == sg.nchunks - 1);
+            if (last && cw == 0 && lane < sg.c1 - sg.a1) lane_add(m, s2, load_elem(sg.ptr, sg.a1 + lane, ELT));
+            const int cur = st;
+            if (++st == STAGES) {
+                st = 0;
+                ph ^= 1u;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hdr->empty[cur]);
+            if (!last) continue;
+            // end of this CTA's segment of row r: the last warp to get here
+            // combines the per-warp partials in warp order and queues the job
+            const int64_t jid = r - r_first;
+            const int ps = (int)(jid % PSLOTS);
+            float lo, hi;
+            unpack2(s2, lo, hi);
+            float sum = lo + hi;
+            warp_combine(m, sum);
+            if (lane == 0) hdr->part[ps][cw] = make_float2(m, sum);
             __syncwarp();
             int old = 0;
             if (lane == 0) {
                 __threadfence_block();
-                old = atomicAdd(&hdr->segcnt[st], 1);
+                old = atomicAdd(&hdr->segcnt[ps], 1);
             }
             old = __shfl_sync(0xffffffffu, old, 0);
             if (old == NCW - 1) {
                 __threadfence_block();
-                float pm = -INFINITY, ps = 0.f;
+                float pm = -INFINITY, pv = 0.f;
                 if (lane < NCW) {
-                    pm = hdr->part[st][lane].x;
-                    ps = hdr->part[st][lane].y;
+                    pm = hdr->part[ps][lane].x;
+                    pv = hdr->part[ps][lane].y;
                 }
-                warp_combine(pm, ps);
+                warp_combine(pm, pv);
                 __syncwarp();
+                if (lane == 0) hdr->segcnt[ps] = 0;
+                const int slot = (int)(jid % QCAP);
+                if (jid >= QCAP &&
+                    !wait_seq(&hdr->freed[slot], (int32_t)(jid - QCAP + 1), &hdr->abort_flag, a.err))
+                    return;
                 if (lane == 0) {
-                    hdr->segcnt[st] = 0;
-                    mbar_arrive(&hdr->empty[st]);
+                    hdr->jobs[slot] = Job{r, pm, pv};
+                    __threadfence_block();
+                    *(volatile int32_t*)&hdr->ready[slot] = (int32_t)(jid + 1);
                 }
-                finish_segment(a, sg, r, r_first, Q, pm, ps);
-            } else {
-                if (lane == 0) mbar_arrive(&hdr->empty[st]);
+                __syncwarp();
             }
             m = -INFINITY;
-            s = 0.f;
+            s2 = pack2(0.f, 0.f);
         }
     }
 }
@@ -768,7 +1003,7 @@ int small_grid(int64_t n) {
 }  // namespace
 
 size_t stream_smem_bytes(int32_t B) {
-    return (size_t)STAGES * STAGE_BYTES + sizeof(SmemHdr) + sizeof(int32_t) * (size_t)(B + 1);
+    return (size_t)RING_BYTES + sizeof(SmemHdr) + sizeof(int32_t) * (size_t)(B + 1);
 }
 
 cudaError_t stream_kernel_setup() {
