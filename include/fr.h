@@ -188,6 +188,30 @@ fr_status fr_beam_read_timing(fr_beam* beam, float* stream_ms, float* select_ms,
 
 void fr_beam_destroy(fr_beam* beam);
 
+/* ------------------------------------------------------------------------ */
+/* Allocation-free row log-sum-exp.  No counterpart in the pages: this is a
+ * library convenience for callers that cannot allocate device memory -- for
+ * example a plugin inside a framework whose allocator owns all device memory,
+ * or a latency-critical path where cudaMalloc's implicit device-wide
+ * synchronisation would stall other streams.  It computes, for each of `rows`
+ * rows, lse[k] = log(sum_v exp(x[k, v])) over v in [0, V), with the streaming
+ * kernel of fr_beam_step (fp32 accumulation), and allocates nothing: its
+ * scratch is a fixed array of about 280 KB that every GPU loading the library
+ * holds until the process exits.
+ *   logits_dev  device [rows, ld] of `dtype`, row k at logits_dev + k*ld elements,
+ *               ld >= V, aligned to the element size
+ *   rows        1 .. 65536 (the scratch's capacity; more -> FR_ERR_INVALID_ARG)
+ *   lse_dev     device float [rows], written
+ * Asynchronous on `stream`.  The first call on a device looks up the
+ * scratch's device address (once per device, with that device current); make
+ * that first call before any stream capture.  All calls share the one
+ * scratch array and leave their contents in it: calls whose work can overlap
+ * on the GPU (different streams, or different host threads) race and must be
+ * serialised by the caller.  A row holding NaN or +inf gets a non-finite
+ * result; no status word is kept. */
+fr_status fr_row_logsumexp_noalloc(const void* logits_dev, int64_t ld, fr_dtype dtype, int32_t rows, int32_t V,
+                                   float* lse_dev, fr_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -105,6 +105,7 @@ struct StreamArgs {
     float2* partial;
     int32_t* row_cnt;
     int32_t* err;
+    float* lse_out;  // log-sum-exp-only instantiation: lse of row (0, k) at lse_out[k]
 };
 
 struct Seg {
@@ -392,9 +393,14 @@ __device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
 
 // The row's log-sum-exp is known: write the scores of the trie children of
 // the row's beam.  One warp.
+template <bool LSE_ONLY>
 __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
     const int lane = threadIdx.x & 31;
     const float lse = m + logf(s);
+    if constexpr (LSE_ONLY) {
+        if (lane == 0) a.lse_out[sg.k] = lse;
+        return;
+    }
     if (!isfinite(lse)) {
         if (lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
     }
@@ -436,13 +442,14 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
 }
 
 // Called by the warp that combined this CTA's partial for row r.
+template <bool LSE_ONLY>
 __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
                                float s) {
     const int lane = threadIdx.x & 31;
     const int64_t fc = (r * a.V) / Q;
     const int64_t lc = ((r + 1) * a.V - 1) / Q;
     if (fc == lc) {
-        finish_row(a, sg, m, s);
+        finish_row<LSE_ONLY>(a, sg, m, s);
         return;
     }
     const int side = (r == r_first) ? 0 : 1;
@@ -469,10 +476,11 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
         combine(M, S, pm, ps);
     }
     if (lane == 0) a.row_cnt[r] = 0;
-    finish_row(a, sg, M, S);
+    finish_row<LSE_ONLY>(a, sg, M, S);
 }
 
-template <bool BF16>
+// LSE_ONLY: the rows' log-sum-exps are the output (no trie, no candidates).
+template <bool BF16, bool LSE_ONLY>
 __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a) {
     constexpr int ELT = BF16 ? 2 : 4;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -580,7 +588,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
                 *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(j + 1);
             }
             const Seg sg = make_seg<ELT>(a, row_start, job.r, bg, eg);
-            finish_segment(a, sg, job.r, r_first, Q, job.m, job.s);
+            finish_segment<LSE_ONLY>(a, sg, job.r, r_first, Q, job.m, job.s);
         }
         return;
     }
@@ -1008,9 +1016,9 @@ size_t stream_smem_bytes(int32_t B) {
 
 cudaError_t stream_kernel_setup() {
     const int max_bytes = (int)stream_smem_bytes(FR_MAX_B);
-    cudaError_t e = cudaFuncSetAttribute(k_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    return cudaFuncSetAttribute(k_stream<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
 }
 
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, const void* logits,
@@ -1034,11 +1042,40 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.partial = buf.partial;
     a.row_cnt = buf.row_cnt;
     a.err = buf.err;
+    a.lse_out = nullptr;
     const size_t smem = stream_smem_bytes(sh.B);
     if (sh.dtype == FR_BF16)
-        k_stream<true><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
+        k_stream<true, false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
     else
-        k_stream<false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
+        k_stream<false, false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
+                           const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
+                           cudaStream_t s) {
+    const int max_bytes = (int)stream_smem_bytes(1);
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_stream<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    if (e != cudaSuccess) return e;
+    StreamArgs a{};
+    a.logits = static_cast<const char*>(logits);
+    a.ld = ld;
+    a.V = V;
+    a.B = 1;  // one "request" whose K = rows beams are all live
+    a.K = rows;
+    a.t = 0;
+    a.elt = dtype == FR_BF16 ? 2 : 4;
+    a.live = live_dev;
+    a.partial = partial;
+    a.row_cnt = row_cnt;
+    a.err = err;
+    a.lse_out = lse_out;
+    if (dtype == FR_BF16)
+        k_stream<true, true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
+    else
+        k_stream<false, true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -31,6 +31,12 @@ cudaError_t stream_kernel_setup();  // raises the kernel's shared-memory limit
 
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
                           const void* logits, int64_t ld, cudaStream_t s);
+// Log-sum-exp of `rows` rows (row k at logits + k*ld elements) into lse_out,
+// with caller-provided scratch: partial [2*grid], row_cnt [rows] (zero on
+// entry, zero again on exit), err [1]; live_dev [1] must hold `rows`.
+cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
+                           const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
+                           cudaStream_t s);
 cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, cudaStream_t s);
 cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s);
 cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,

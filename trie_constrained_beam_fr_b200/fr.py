@@ -56,6 +56,7 @@ FR_FUNCS = [
     ("fr_beam_set_timing", _I32, [_VP, _I32]),
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
+    ("fr_row_logsumexp_noalloc", _I32, [_VP, _I64, _I32, _I32, _I32, _VP, _VP]),
 ]
 FR_GEN_FUNCS = [
     ("fr_gen_hash_logits", _I32, [_U64, _I64, _I32, _I32, _I32, _I64, _I32, _VP, _I32, _I32, _VP, _VP, _VP]),
@@ -274,6 +275,17 @@ def fr_beam_read_timing(beam, max_steps: int = 4096):
 
 def fr_beam_destroy(beam) -> None:
     libfr().fr_beam_destroy(beam)
+
+
+def fr_row_logsumexp_noalloc(logits: torch.Tensor, rows: int, V: int, lse: torch.Tensor,
+                             ld: Optional[int] = None, stream=None) -> None:
+    """Allocation-free log-sum-exp of `rows` logits rows (see include/fr.h)."""
+    if lse.dtype != torch.float32 or not lse.is_cuda:
+        raise ValueError("lse must be a float32 CUDA tensor")
+    if ld is None:
+        ld = logits.stride(-2) if logits.dim() >= 2 else V
+    _check(libfr().fr_row_logsumexp_noalloc(_dev_ptr(logits), int(ld), _dtype_code(logits.dtype), int(rows),
+                                            int(V), _dev_ptr(lse), _stream(stream)), "fr_row_logsumexp_noalloc")
 
 
 # ---------------------------------------------------------------------------
