@@ -55,6 +55,30 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def rank_requests(rank: int, world: int, B: int):
+    """Requests are independent, so ranks shard them: rank r decodes the
+    global requests r*B .. r*B+B-1 (the hash logits take the global index)."""
+    if not (0 <= rank < world) or B < 1:
+        raise ValueError("bad rank layout")
+    return rank * B, B
+
+
+def max_over_ranks(x: float, world: int, dist=None, device=None) -> float:
+    """The job's time is its slowest rank's (one all-reduce, not on the data path)."""
+    if world == 1:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, candidates_per_decode: int, decodes: int, elapsed_ms: float) -> float:
+    """Whole-job candidates/s: every rank's decodes over the slowest rank's time."""
+    return world * candidates_per_decode * decodes / (elapsed_ms / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -230,12 +254,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, world, dist, dev)
 
     w = synth.WORKLOADS[args.config]
     if args.batch:
@@ -243,7 +263,7 @@ def main():
     B, K, D, V = w.B, w.K, w.depth, w.V
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     elt = w.elt_size
-    b_offset = rank * B  # each rank decodes its own requests
+    b_offset, _ = rank_requests(rank, world, B)  # each rank decodes its own requests
 
     sids_np = synth.workload_catalog(w)
     sids = torch.from_numpy(sids_np).to(dev)
@@ -302,14 +322,14 @@ def main():
         torch.cuda.synchronize()
     barrier()
     fr.fr_beam_set_timing(beam, False)
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    elapsed_ms = slowest(t_start.elapsed_time(t_end))
     stream_ms, select_ms = fr.fr_beam_read_timing(beam)
     st = fr.fr_beam_status(beam)
     if st != fr.FR_OK:
         raise RuntimeError("timed decode failed: " + fr.fr_status_string(st))
     ms_per_decode = elapsed_ms / args.steps
     cands_per_decode = B * K * D
-    value = world * cands_per_decode * args.steps / (elapsed_ms / 1e3)
+    value = job_throughput(world, cands_per_decode, args.steps, elapsed_ms)
 
     # roofline of the dominant kernel: the streaming log-sum-exp / candidate kernel
     peak, peak_kind = measured_peaks()
@@ -367,7 +387,7 @@ def main():
         b_.record()
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(a.elapsed_time(b_)) / args.e2e_steps
+        e2e_ms = slowest(a.elapsed_time(b_)) / args.e2e_steps
         e2e = {"value": world * cands_per_decode / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": D * B * K * V * elt,
                "d2h_bytes_per_step": B * K * D * 4 + B * K * 4 + B * K * 4,
