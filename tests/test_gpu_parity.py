@@ -38,6 +38,10 @@ SMALL = {
                            dtype="f32", seed=7, catalog_seed=7),
     "skewed_small": W("skewed_small", B=2, K=128, depth=3, C=256, V=5000, sid_base=1000, n_items=30000,
                       dtype="f32", seed=8, catalog_seed=8, zipf_levels=2),
+    # K x max fan-out = 1024 x 1024 candidates: beyond what a 16-CTA cluster
+    # holds in shared memory, so the selection reads the candidates from L2
+    "k1024_wide_fanout": W("k1024_wide_fanout", B=2, K=1024, depth=2, C=1024, V=2100, sid_base=30,
+                           n_items=60000, dtype="bf16", seed=10, catalog_seed=10),
 }
 
 

@@ -13,6 +13,7 @@ struct fr_trie {
     int32_t codebook[FR_MAX_DEPTH] = {};
     int64_t nodes[FR_MAX_DEPTH + 1] = {};
     int32_t max_fanout = 0;
+    int32_t level_fanout[FR_MAX_DEPTH] = {};  // largest child count of a level-l node
     int32_t device = 0;
     int32_t* child_off[FR_MAX_DEPTH] = {};
     int32_t* code[FR_MAX_DEPTH + 1] = {};

@@ -30,6 +30,7 @@
 //
 // Every wait on an mbarrier is bounded: after 2 s the kernel records
 // FR_ERR_DEVICE in the beam's status word and returns.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -693,6 +694,7 @@ struct SelectArgs {
     int32_t* parent_out;
     int32_t* token_out;
     int32_t* err;
+    int32_t key_cap;  // cluster select: keys each CTA's shared memory holds
 };
 
 __device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t* out_or) {
@@ -730,6 +732,93 @@ __device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, 
     if (j < K) cand_off_row[j] = e;
     if (j == 0) cand_off_row[K] = tot;
 }
+
+// Sorts the Kp winners in sel (descending (key, ~slot), so score descending,
+// then slot ascending) and writes the request's next state: the reorder
+// gathers and the next step's candidate offsets.  All threads of the block
+// (blockDim.x >= K) call it.
+__device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, int Kp,
+                                 unsigned long long* sel) {
+    const int tid = threadIdx.x;
+    const int K = a.K, D = a.D, t = a.t;
+    int P = 1;
+    while (P < Kp) P <<= 1;
+    for (int i = Kp + tid; i < P; i += blockDim.x) sel[i] = 0ull;
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const unsigned long long x = sel[i], y = sel[ixj];
+                    const bool swap = ((i & k) == 0) ? (x < y) : (x > y);
+                    if (swap) {
+                        sel[i] = y;
+                        sel[ixj] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // emit survivors (thread j = slot j)
+    const int j = tid;
+    int32_t child = -1;
+    if (j < K) {
+        const int64_t oj = (int64_t)b * K + j;
+        if (j < Kp) {
+            const unsigned long long v = sel[j];
+            const uint32_t key = (uint32_t)(v >> 32);
+            const int32_t slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
+            int lo = 0, hi = live - 1;  // parent: last k with s_off[k] <= slot
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
+            }
+            const int k = lo;
+            const int64_t ok = (int64_t)b * K + k;
+            const int32_t np = a.cur.node[ok];
+            int32_t tok = -1;
+            if (np >= 0 && np < a.trie.nodes[t]) {
+                child = a.trie.child_off[t][np] + (slot - s_off[k]);
+                if (child >= 0 && child < a.trie.nodes[t + 1]) {
+                    tok = a.trie.tok_base[t] + a.trie.code[t + 1][child];
+                } else {
+                    child = -1;
+                }
+            }
+            if (child < 0) set_error(a.err, FR_ERR_DEVICE);
+            a.nxt.node[oj] = child;
+            a.nxt.score[oj] = key_to_float(key);
+            a.nxt.kv[oj] = a.cur.kv[ok];
+            a.parent_out[oj] = k;
+            a.token_out[oj] = tok;
+            for (int l = 0; l < D; ++l)
+                a.nxt.prefix[oj * D + l] = (l < t) ? a.cur.prefix[ok * D + l] : (l == t ? tok : -1);
+        } else {
+            a.nxt.node[oj] = -1;
+            a.nxt.score[oj] = -INFINITY;
+            a.nxt.kv[oj] = -1;
+            a.parent_out[oj] = -1;
+            a.token_out[oj] = -1;
+            for (int l = 0; l < D; ++l) a.nxt.prefix[oj * D + l] = -1;
+        }
+    }
+    if (tid == 0) a.nxt.live[b] = Kp;
+    if (t + 1 < D) {
+        // node ids of the survivors are in registers of threads 0..Kp-1
+        const int jj = threadIdx.x;
+        int cnt = 0;
+        if (jj < Kp && child >= 0) cnt = a.trie.child_off[t + 1][child + 1] - a.trie.child_off[t + 1][child];
+        int tot;
+        const int e = block_excl_scan(cnt, &tot);
+        int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
+        if (jj < K) row[jj] = e;
+        if (jj == 0) row[K] = tot;
+    }
+}
+
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     __shared__ int32_t s_off[FR_MAX_K + 1];
@@ -841,84 +930,181 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
         }
         __syncthreads();
         if (tid == 0 && s_misc[3] != Kp) set_error(a.err, FR_ERR_DEVICE);
-        // bitonic sort, descending, over the next power of two
-        int P = 1;
-        while (P < Kp) P <<= 1;
-        for (int i = Kp + tid; i < P; i += SEL_THREADS) sel[i] = 0ull;
-        __syncthreads();
-        for (int k = 2; k <= P; k <<= 1) {
-            for (int j = k >> 1; j > 0; j >>= 1) {
-                for (int i = tid; i < P; i += SEL_THREADS) {
-                    const int ixj = i ^ j;
-                    if (ixj > i) {
-                        const unsigned long long x = sel[i], y = sel[ixj];
-                        const bool swap = ((i & k) == 0) ? (x < y) : (x > y);
-                        if (swap) {
-                            sel[i] = y;
-                            sel[ixj] = x;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-        }
+    }
+    select_sort_emit(a, b, live, s_off, Kp, sel);
+}
+
+// ---------------------------------------------------------------------------
+// Selection with one thread-block cluster per request.  Each CTA of the
+// cluster holds a contiguous slice of the request's candidates in shared
+// memory as order-preserving keys, loaded once; the bits shared by every key
+// are skipped (cluster-wide AND/OR), and each 12-bit radix pass histograms the
+// slices locally, after which every CTA reads all peers' histograms through
+// distributed shared memory and derives the same threshold digit.  Winners go
+// straight into the leader CTA's array (DSMEM atomics); keys equal to the
+// threshold are taken in slot order (slices are contiguous in slot order, so
+// each CTA starts from the count of equal keys in the slices before it).  The
+// leader sorts and emits.  Every CTA runs the same sequence of cluster
+// barriers: their number depends only on cluster-wide values.
+
+namespace cg = cooperative_groups;
+constexpr int CSEL_MAXKEYS = 40960;  // keys per CTA (160 KB of shared memory)
+
+__global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectArgs a) {
+    cg::cluster_group cl = cg::this_cluster();
+    extern __shared__ __align__(16) uint32_t keys[];
+    __shared__ __align__(16) int32_t hist[2][HBINS];
+    __shared__ unsigned long long sel[FR_MAX_K];
+    __shared__ int32_t s_off[FR_MAX_K + 1];
+    __shared__ uint32_t red[64];
+    __shared__ int32_t s_misc[8];
+    __shared__ uint32_t s_ao[2];
+    const int CS = (int)cl.num_blocks();
+    const int c = (int)cl.block_rank();
+    const int b = blockIdx.x / CS;
+    const int tid = threadIdx.x;
+    const int K = a.K;
+    const int live = min(max(a.cur.live[b], 0), K);
+    const int32_t* off_row = a.cur.cand_off + (int64_t)b * (K + 1);
+    int n = off_row[live];
+    if (n < 0 || (int64_t)n > a.cand_stride || (n + CS - 1) / CS > a.key_cap) {
+        if (tid == 0 && c == 0) set_error(a.err, FR_ERR_DEVICE);
+        n = 0;
+    }
+    const int Kp = min(K, n);
+    const int S = (n + CS - 1) / CS;
+    const int lo = min(n, c * S), hi = min(n, lo + S);
+    const int cnt = hi - lo;
+    if (c == 0) {
+        for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = off_row[i];
+        if (tid == 0) s_misc[0] = 0;  // the leader's winner count
+    }
+    const float* cb = a.cand + (int64_t)b * a.cand_stride + lo;
+    uint32_t va = 0xFFFFFFFFu, vo = 0u;
+    for (int i = tid; i < cnt; i += SEL_THREADS) {
+        const uint32_t k = float_to_key(cb[i]);
+        keys[i] = k;
+        va &= k;
+        vo |= k;
+    }
+    uint32_t VO;
+    const uint32_t VA = block_and_or(va, vo, red, &VO);
+    if (tid == 0) {
+        s_ao[0] = VA;
+        s_ao[1] = VO;
+    }
+    cl.sync();
+    uint32_t GA = 0xFFFFFFFFu, GO = 0u;
+    for (int r = 0; r < CS; ++r) {
+        const uint32_t* p = cl.map_shared_rank(s_ao, r);
+        GA &= p[0];
+        GO |= p[1];
     }
 
-    // emit survivors (thread j = slot j)
-    const int j = tid;
-    int32_t child = -1;
-    if (j < K) {
-        const int64_t oj = (int64_t)b * K + j;
-        if (j < Kp) {
-            const unsigned long long v = sel[j];
-            const uint32_t key = (uint32_t)(v >> 32);
-            const int32_t slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
-            int lo = 0, hi = live - 1;  // parent: last k with s_off[k] <= slot
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
-            }
-            const int k = lo;
-            const int64_t ok = (int64_t)b * K + k;
-            const int32_t np = a.cur.node[ok];
-            int32_t tok = -1;
-            if (np >= 0 && np < a.trie.nodes[t]) {
-                child = a.trie.child_off[t][np] + (slot - s_off[k]);
-                if (child >= 0 && child < a.trie.nodes[t + 1]) {
-                    tok = a.trie.tok_base[t] + a.trie.code[t + 1][child];
-                } else {
-                    child = -1;
-                }
-            }
-            if (child < 0) set_error(a.err, FR_ERR_DEVICE);
-            a.nxt.node[oj] = child;
-            a.nxt.score[oj] = key_to_float(key);
-            a.nxt.kv[oj] = a.cur.kv[ok];
-            a.parent_out[oj] = k;
-            a.token_out[oj] = tok;
-            for (int l = 0; l < D; ++l)
-                a.nxt.prefix[oj * D + l] = (l < t) ? a.cur.prefix[ok * D + l] : (l == t ? tok : -1);
+    uint32_t T = 0u;
+    int eq_needed = 0, count_eq = 0, eq_before = 0;
+    if (Kp > 0) {
+        const uint32_t diff = GA ^ GO;
+        if (diff == 0u) {
+            T = GA;
+            eq_needed = Kp;
+            count_eq = n;
+            eq_before = lo;
         } else {
-            a.nxt.node[oj] = -1;
-            a.nxt.score[oj] = -INFINITY;
-            a.nxt.kv[oj] = -1;
-            a.parent_out[oj] = -1;
-            a.token_out[oj] = -1;
-            for (int l = 0; l < D; ++l) a.nxt.prefix[oj * D + l] = -1;
+            int lob = 32 - __clz(diff);
+            uint32_t prefix = (lob == 32) ? 0u : (GA & (0xFFFFFFFFu << lob));
+            int krem = Kp;
+            int pass = 0;
+            while (lob > 0) {
+                const int width = min(HBITS, lob);
+                const int shift = lob - width;
+                const uint32_t dmask = (1u << width) - 1u;
+                int32_t* h = hist[pass & 1];
+                for (int i = tid; i < HBINS; i += SEL_THREADS) h[i] = 0;
+                __syncthreads();
+                const uint64_t want = (uint64_t)prefix >> lob;
+                for (int i = tid; i < cnt; i += SEL_THREADS) {
+                    const uint32_t k = keys[i];
+                    if (((uint64_t)k >> lob) == want) atomicAdd(&h[(k >> shift) & dmask], 1);
+                }
+                __syncthreads();
+                cl.sync();
+                int g4[4] = {0, 0, 0, 0};
+                for (int r = 0; r < CS; ++r) {
+                    const int4 v = *reinterpret_cast<const int4*>(cl.map_shared_rank(h, r) + tid * 4);
+                    g4[0] += v.x;
+                    g4[1] += v.y;
+                    g4[2] += v.z;
+                    g4[3] += v.w;
+                }
+                const int tsum = g4[0] + g4[1] + g4[2] + g4[3];
+                int tot;
+                const int excl = block_excl_scan(tsum, &tot);
+                int cum = tot - excl - tsum;  // keys in the bins above this thread's
+#pragma unroll
+                for (int q = 3; q >= 0; --q) {
+                    if (cum < krem && cum + g4[q] >= krem) {
+                        s_misc[1] = tid * 4 + q;
+                        s_misc[2] = cum;
+                        s_misc[3] = g4[q];
+                    }
+                    cum += g4[q];
+                }
+                __syncthreads();
+                const int d = s_misc[1];
+                krem -= s_misc[2];
+                count_eq = s_misc[3];
+                if (tid == 0) {
+                    int before = 0;
+                    for (int r = 0; r < c; ++r) before += cl.map_shared_rank(h, r)[d];
+                    s_misc[4] = before;
+                }
+                prefix |= (uint32_t)d << shift;
+                lob = shift;
+                ++pass;
+                __syncthreads();
+                eq_before = s_misc[4];
+            }
+            T = prefix;
+            eq_needed = krem;
         }
     }
-    if (tid == 0) a.nxt.live[b] = Kp;
-    if (t + 1 < D) {
-        // node ids of the survivors are in registers of threads 0..Kp-1
-        const int jj = threadIdx.x;
-        int cnt = 0;
-        if (jj < Kp && child >= 0) cnt = a.trie.child_off[t + 1][child + 1] - a.trie.child_off[t + 1][child];
-        int tot;
-        const int e = block_excl_scan(cnt, &tot);
-        int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
-        if (jj < K) row[jj] = e;
-        if (jj == 0) row[K] = tot;
+    // collect: every key > T, and the keys == T whose slot-order rank among
+    // the equal keys is below eq_needed
+    unsigned long long* lsel = cl.map_shared_rank(sel, 0);
+    int32_t* lcnt = cl.map_shared_rank(&s_misc[0], 0);
+    if (Kp > 0) {
+        const bool all_eq = eq_needed >= count_eq;
+        const bool no_eq = !all_eq && eq_before >= eq_needed;
+        if (all_eq || no_eq) {
+            for (int i = tid; i < cnt; i += SEL_THREADS) {
+                const uint32_t k = keys[i];
+                if (k > T || (all_eq && k == T)) {
+                    const int p = atomicAdd(lcnt, 1);
+                    if (p < FR_MAX_K) lsel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i));
+                }
+            }
+        } else {
+            int run = eq_before;
+            for (int base = 0; base < cnt; base += SEL_THREADS) {
+                const int i = base + tid;
+                const uint32_t k = i < cnt ? keys[i] : 0u;
+                const bool gt = i < cnt && k > T;
+                const bool eq = i < cnt && k == T;
+                int tot;
+                const int r = block_excl_scan(eq ? 1 : 0, &tot);
+                if (gt || (eq && run + r < eq_needed)) {
+                    const int p = atomicAdd(lcnt, 1);
+                    if (p < FR_MAX_K) lsel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i));
+                }
+                run += tot;
+            }
+        }
     }
+    cl.sync();
+    if (c != 0) return;
+    if (tid == 0 && s_misc[0] != Kp) set_error(a.err, FR_ERR_DEVICE);
+    select_sort_emit(a, b, live, s_off, Kp, sel);
 }
 
 // ---------------------------------------------------------------------------
@@ -1093,8 +1279,64 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
     a.parent_out = buf.parent;
     a.token_out = buf.token;
     a.err = buf.err;
-    k_select<<<sh.B, SEL_THREADS, 0, s>>>(a);
-    return cudaGetLastError();
+    const int cs = sh.sel_cluster[t];
+    if (cs <= 0) {
+        k_select<<<sh.B, SEL_THREADS, 0, s>>>(a);
+        return cudaGetLastError();
+    }
+    a.key_cap = (int32_t)((sh.sel_bound[t] + cs - 1) / cs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sh.B * cs));
+    cfg.blockDim = dim3(SEL_THREADS);
+    cfg.dynamicSmemBytes = (size_t)a.key_cap * sizeof(uint32_t);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_select_cluster, a);
+}
+
+int select_cluster_size(int32_t B, int64_t bound, int32_t sms) {
+    // Few candidates: one CTA per request is quickest (no cluster barriers).
+    // Very many: they do not fit a small cluster's shared memory; one CTA per
+    // request reads them from L2.  In between, a cluster of up to 4 CTAs per
+    // request, as long as every request's cluster runs in the same wave.
+    constexpr int64_t SMALL_BOUND = 8192;
+    constexpr int MAX_CS = 4;
+    if (bound <= SMALL_BOUND) return 0;
+    int need = 1;
+    while ((bound + need - 1) / need > CSEL_MAXKEYS) need <<= 1;
+    if (need > MAX_CS) return 0;
+    int fill = 1;
+    while (fill * 2 * B <= sms && fill < MAX_CS) fill <<= 1;
+    const int cs = need > fill ? need : fill;
+    if (cs < 2 || (int64_t)B * cs > sms) return 0;
+    if (cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CSEL_MAXKEYS * (int)sizeof(uint32_t)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(B * cs));
+    cfg.blockDim = dim3(SEL_THREADS);
+    cfg.dynamicSmemBytes = (size_t)((bound + cs - 1) / cs) * sizeof(uint32_t);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, k_select_cluster, &cfg) != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    return cs;
 }
 
 cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s) {

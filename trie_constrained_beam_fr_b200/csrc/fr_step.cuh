@@ -23,7 +23,13 @@ struct StepShape {
     int32_t B, K, V, D;
     int32_t dtype;  // fr_dtype
     int32_t grid;   // CTAs of the streaming kernel
+    int32_t sel_cluster[FR_MAX_DEPTH];  // per step: CTAs per request of the cluster select (0: one CTA)
+    int64_t sel_bound[FR_MAX_DEPTH];    // per step: most candidates a request can have
 };
+
+// Cluster size of the selection for a step whose requests have at most
+// `bound` candidates (0 = the single-CTA kernel).
+int select_cluster_size(int32_t B, int64_t bound, int32_t sms);
 
 // Streaming kernel: dynamic shared memory it needs for B requests.
 size_t stream_smem_bytes(int32_t B);

@@ -395,14 +395,16 @@ static fr_status trie_build_impl(const int32_t* sids, int64_t n, int32_t depth, 
     }
 
     // Largest child count.
-    FR_CUDA_TRY(cudaMemsetAsync(dev_words + 4, 0, sizeof(int32_t), s));
+    int32_t* fan;
+    FR_CUDA_TRY(tmp.alloc(&fan, FR_MAX_DEPTH));
+    FR_CUDA_TRY(cudaMemsetAsync(fan, 0, sizeof(int32_t) * FR_MAX_DEPTH, s));
     for (int l = 0; l < depth; ++l)
-        k_max_fanout<<<grid_for(t->nodes[l], 256), 256, 0, s>>>(t->child_off[l], t->nodes[l], dev_words + 4);
+        k_max_fanout<<<grid_for(t->nodes[l], 256), 256, 0, s>>>(t->child_off[l], t->nodes[l], fan + l);
     FR_CUDA_TRY(cudaGetLastError());
-    int32_t mf = 0;
-    FR_CUDA_TRY(cudaMemcpyAsync(&mf, dev_words + 4, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    FR_CUDA_TRY(cudaMemcpyAsync(t->level_fanout, fan, sizeof(int32_t) * depth, cudaMemcpyDeviceToHost, s));
     FR_CUDA_TRY(cudaStreamSynchronize(s));
-    t->max_fanout = mf;
+    t->max_fanout = 0;
+    for (int l = 0; l < depth; ++l) t->max_fanout = std::max(t->max_fanout, t->level_fanout[l]);
 
     // Device view.
     t->dev.depth = depth;
