@@ -22,6 +22,10 @@ _LIB_PATH = os.path.join(_OUT_DIR, "liboracle.so")
 # The mutation test loads deliberately broken copies of the oracle through this.
 _LIB_OVERRIDE = os.environ.get("FR_ORACLE_LIB")
 
+NORM_FULL = 0
+NORM_SID_RANGE = 1
+NORM_CANDIDATES = 2
+
 MODE_HASH_F32 = 0
 MODE_HASH_BF16 = 1
 MODE_CONST = 2
@@ -50,7 +54,7 @@ class _Cfg(ctypes.Structure):
                 ("depth", ctypes.c_int32), ("sid_base", ctypes.c_int32),
                 ("codebook", ctypes.c_int32 * 16), ("mode", ctypes.c_int32),
                 ("const_logit", ctypes.c_float), ("seed", ctypes.c_uint64),
-                ("b_offset", ctypes.c_int64)]
+                ("b_offset", ctypes.c_int64), ("norm", ctypes.c_int32)]
 
 
 _lib = None
@@ -139,19 +143,20 @@ class Config:
     const_logit: float = 0.0
     seed: int = 0
     b_offset: int = 0
+    norm: int = NORM_FULL
 
     @classmethod
     def from_workload(cls, w, mode: Optional[int] = None, B: Optional[int] = None,
-                      b_offset: int = 0) -> "Config":
+                      b_offset: int = 0, norm: int = NORM_FULL) -> "Config":
         if mode is None:
             mode = MODE_HASH_BF16 if w.dtype == "bf16" else MODE_HASH_F32
         return cls(B=w.B if B is None else B, K=w.K, V=w.V, depth=w.depth, sid_base=w.sid_base,
-                   codebook=list(w.codebook_sizes), mode=mode, seed=w.seed, b_offset=b_offset)
+                   codebook=list(w.codebook_sizes), mode=mode, seed=w.seed, b_offset=b_offset, norm=norm)
 
     def c(self) -> _Cfg:
         cb = (ctypes.c_int32 * 16)(*([int(x) for x in self.codebook] + [0] * (16 - len(self.codebook))))
         return _Cfg(self.B, self.K, self.V, self.depth, self.sid_base, cb, self.mode,
-                    self.const_logit, self.seed & 0xFFFFFFFFFFFFFFFF, self.b_offset)
+                    self.const_logit, self.seed & 0xFFFFFFFFFFFFFFFF, self.b_offset, self.norm)
 
     def token_base(self, level: int) -> int:
         return self.sid_base + int(sum(self.codebook[:level]))

@@ -51,6 +51,18 @@
 #define ORC_ERR_OOM 4
 #define ORC_ERR_NOT_IN_CATALOG 5
 
+/* Normalisation sets of the step's log-softmax:
+ *  FULL       the whole vocabulary (the default reading);
+ *  SID_RANGE  the SID token range [sid_base, sid_base + C_0 + ... + C_{D-1})
+ *             ("flashrec 0.1.1 METADATA", §Features/Decoding: lm_head is
+ *             evaluated only over the SID token range);
+ *  CANDIDATES the beam's allowed children ("Qwen-2.5-1B-RLCD-Fast",
+ *             §Parallel Evaluation step 4: probabilities over the candidate
+ *             slice), at temperature 1. */
+#define ORC_NORM_FULL 0
+#define ORC_NORM_SID_RANGE 1
+#define ORC_NORM_CANDIDATES 2
+
 #define ORC_MODE_HASH_F32 0
 #define ORC_MODE_HASH_BF16 1
 #define ORC_MODE_CONST 2
@@ -109,6 +121,7 @@ typedef struct {
     float const_logit;  /* ORC_MODE_CONST */
     uint64_t seed;
     int64_t b_offset;   /* request index of local request 0 in the hash */
+    int32_t norm;       /* ORC_NORM_*: the set the log-softmax normalises over */
 } orc_cfg;
 
 static int32_t level_token_base(const orc_cfg* cfg, int32_t level) {
@@ -138,6 +151,16 @@ double orc_row_lse(const float* x, int64_t V) {
         if ((double)x[v] > m) m = (double)x[v];
     double s = 0.0;
     for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);
+    return m + log(s);
+}
+
+/* log of sum exp(x[idx[i]]) over the n given columns, in double. */
+double orc_subset_lse(const float* x, const int32_t* idx, int32_t n) {
+    double m = -INFINITY;
+    for (int32_t i = 0; i < n; ++i)
+        if ((double)x[idx[i]] > m) m = (double)x[idx[i]];
+    double s = 0.0;
+    for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);
     return m + log(s);
 }
 
@@ -318,6 +341,7 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     float* row = (float*)malloc(sizeof(float) * (size_t)cfg->V);
     int32_t cap = cfg->codebook[t];
     int32_t* kids = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+    int32_t* slice = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
     orc_cand* cand = (orc_cand*)malloc(sizeof(orc_cand) * (size_t)(live > 0 ? live : 1) * cap);
     int32_t tokens[16];
     int64_t nc = 0;
@@ -327,8 +351,18 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
         double t0 = now_seconds();
         orc_fill_row(cfg, b, tokens, t, row);
         g_gen_seconds += now_seconds() - t0;
-        double lse = orc_row_lse(row, cfg->V);
         int32_t nk = orc_children(cat, prefix + k * D, t, kids, cap);
+        double lse;
+        if (cfg->norm == ORC_NORM_SID_RANGE) {
+            int32_t span = 0;
+            for (int32_t l = 0; l < D; ++l) span += cfg->codebook[l];
+            lse = orc_row_lse(row + cfg->sid_base, span);
+        } else if (cfg->norm == ORC_NORM_CANDIDATES) {
+            for (int32_t i = 0; i < nk; ++i) slice[i] = tok_base + kids[i];
+            lse = orc_subset_lse(row, slice, nk);
+        } else {
+            lse = orc_row_lse(row, cfg->V);
+        }
         for (int32_t i = 0; i < nk; ++i) {
             int32_t tok = tok_base + kids[i];
             cand[nc].score = score[k] + ((double)row[tok] - lse);
@@ -358,6 +392,7 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     }
     free(row);
     free(kids);
+    free(slice);
     free(cand);
     return nlive;
 }

@@ -42,6 +42,10 @@ MUTANTS = {
     "logit_offset": ("return (float)(u >> 40) * 0x1p-21f - 4.0f;",
                      "return (float)(u >> 40) * 0x1p-21f - 3.0f;"),
     "prefix_hash_seed": ("uint64_t h = 0x243F6A8885A308D3ULL;", "uint64_t h = 0;"),
+    "sid_range_short": ("for (int32_t l = 0; l < D; ++l) span += cfg->codebook[l];",
+                        "for (int32_t l = 0; l < D - 1; ++l) span += cfg->codebook[l];"),
+    "candidate_slice_shifted": ("for (int32_t i = 0; i < nk; ++i) slice[i] = tok_base + kids[i];",
+                                "for (int32_t i = 0; i < nk; ++i) slice[i] = tok_base + kids[i] + 1;"),
     "token_base_skips_level": ("for (int32_t i = 0; i < level; ++i) base += cfg->codebook[i];",
                                "for (int32_t i = 1; i < level; ++i) base += cfg->codebook[i];"),
 }

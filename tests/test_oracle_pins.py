@@ -171,17 +171,28 @@ def _tiny_cfg(K, n_items, mode=oracle.MODE_HASH_F32, seed=0, V=64, C=16, D=3, si
 
 def _brute_force(cfg, sids, b=0):
     """Every catalog SID scored by the sum over levels of its token's
-    log-probability under the row its prefix sees (scipy logsumexp)."""
+    log-probability under the row its prefix sees (scipy logsumexp over the
+    normalisation set: the vocabulary, the SID token range, or the prefix's
+    catalog children)."""
+    tuples = [tuple(x) for x in np.unique(sids, axis=0).tolist()]
     rows = {}
     out = []
-    for sid in np.unique(sids, axis=0).tolist():
+    span = int(sum(cfg.codebook))
+    for sid in tuples:
         s = 0.0
         for t in range(cfg.depth):
             key = tuple(sid[:t])
             if key not in rows:
                 toks = [cfg.token_base(l) + sid[l] for l in range(t)]
-                r = oracle.fill_row(cfg, b, toks)
-                rows[key] = (r, float(logsumexp(r.astype(np.float64))))
+                r = oracle.fill_row(cfg, b, toks).astype(np.float64)
+                if cfg.norm == oracle.NORM_SID_RANGE:
+                    lse = float(logsumexp(r[cfg.sid_base: cfg.sid_base + span]))
+                elif cfg.norm == oracle.NORM_CANDIDATES:
+                    kids = sorted({q[t] for q in tuples if q[:t] == key})
+                    lse = float(logsumexp(r[[cfg.token_base(t) + c for c in kids]]))
+                else:
+                    lse = float(logsumexp(r))
+                rows[key] = (r, lse)
             r, lse = rows[key]
             s = s + (float(r[cfg.token_base(t) + sid[t]]) - lse)
         out.append((s, tuple(sid)))
@@ -303,3 +314,45 @@ def test_requests_are_independent():
     r = oracle.decode(one, cat)
     np.testing.assert_array_equal(r.sids[0], full.sids[2])
     np.testing.assert_array_equal(r.scores[0], full.scores[2])
+
+
+@pytest.mark.parametrize("norm", [oracle.NORM_SID_RANGE, oracle.NORM_CANDIDATES])
+@pytest.mark.parametrize("mode", [oracle.MODE_HASH_F32, oracle.MODE_HASH_BF16])
+def test_bruteforce_other_normalisations(norm, mode):
+    w, sids, cfg = _tiny_cfg(600, 500, mode, seed=4, catalog_seed=4)
+    cfg.norm = norm
+    res = oracle.decode(cfg, oracle.Catalog(sids, w.codebook_sizes))
+    bf = _brute_force(cfg, sids)
+    n = len(bf)
+    want = np.array([s for s, _ in bf])
+    np.testing.assert_allclose(res.scores[0, :n], want, atol=1e-9, rtol=0)
+    assert {tuple(x) for x in res.sids[0, :n].tolist()} == {sid for _, sid in bf}
+
+
+def test_candidate_slice_probabilities_sum_to_one():
+    """Over the candidate slice every level's conditional distribution sums to
+    one over the allowed children, so when nothing is pruned the probabilities
+    of all catalog SIDs sum to exactly one."""
+    for seed, n_items in [(0, 500), (3, 50), (5, 300)]:
+        w, sids, cfg = _tiny_cfg(600, n_items, oracle.MODE_HASH_F32, seed=seed, catalog_seed=seed)
+        cfg.norm = oracle.NORM_CANDIDATES
+        res = oracle.decode(cfg, oracle.Catalog(sids, w.codebook_sizes))
+        n = int(res.step_live[-1, 0])
+        assert n == len(np.unique(sids, axis=0))
+        assert float(np.exp(res.scores[0, :n]).sum()) == pytest.approx(1.0, abs=1e-12)
+        # the SID-range normalisation puts the same SIDs below one (other SID tokens share the mass)
+        cfg.norm = oracle.NORM_SID_RANGE
+        res2 = oracle.decode(cfg, oracle.Catalog(sids, w.codebook_sizes))
+        assert 0.0 < float(np.exp(res2.scores[0, :n]).sum()) < 1.0
+
+
+def test_greedy_path_does_not_depend_on_the_normalisation():
+    """The normaliser is one constant per row, so the best child -- and the
+    greedy SID -- is the same for every normalisation set."""
+    w, sids, cfg = _tiny_cfg(1, 500, oracle.MODE_HASH_BF16, seed=6, V=300, C=64, sid_base=50, catalog_seed=6)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    paths = []
+    for norm in (oracle.NORM_FULL, oracle.NORM_SID_RANGE, oracle.NORM_CANDIDATES):
+        cfg.norm = norm
+        paths.append(oracle.decode(cfg, cat).sids[0, 0].tolist())
+    assert paths[0] == paths[1] == paths[2]
