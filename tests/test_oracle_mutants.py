@@ -19,7 +19,10 @@ SRC = os.path.join(ROOT, "oracle", "fr_oracle.c")
 MUTANTS = {
     "score_sign": ("cand[nc].score = score[k] + ((double)row[tok] - lse);",
                    "cand[nc].score = score[k] - ((double)row[tok] - lse);"),
-    "lse_drops_max": ("return m + log(s);", "return log(s);"),
+    "lse_drops_max": ("for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);\n    return m + log(s);",
+                      "for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);\n    return log(s);"),
+    "subset_lse_drops_max": ("for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);\n    return m + log(s);",
+                             "for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);\n    return log(s);"),
     "lse_max_wrong_way": ("if ((double)x[v] > m) m = (double)x[v];", "if ((double)x[v] < m) m = (double)x[v];"),
     "order_ascending": ("if (a->score != b->score) return a->score > b->score ? -1 : 1;",
                         "if (a->score != b->score) return a->score < b->score ? -1 : 1;"),
