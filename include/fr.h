@@ -61,6 +61,13 @@ typedef enum {
 
 typedef enum { FR_F32 = 0, FR_BF16 = 1 } fr_dtype;
 
+/* The set each live row's log-softmax normalises over. */
+typedef enum {
+    FR_NORM_FULL = 0,       /* the whole vocabulary [0, V) (default) */
+    FR_NORM_SID_RANGE = 1,  /* the SID token range [sid_base, sid_base + C_0 + ... + C_{D-1}) */
+    FR_NORM_CANDIDATES = 2  /* the beam's allowed children (the candidate slice) */
+} fr_norm;
+
 typedef struct fr_trie fr_trie; /* opaque, library-owned */
 typedef struct fr_beam fr_beam; /* opaque, library-owned */
 
@@ -176,6 +183,15 @@ fr_status fr_beam_get_state(fr_beam* beam, int32_t* steps_done, int32_t* live_ho
 fr_status fr_beam_set_state(fr_beam* beam, int32_t steps_done, const int32_t* live_host,
                             const int32_t* prefix_host, const float* score_host,
                             const int32_t* kv_host, fr_stream stream);
+
+/* Normalisation set of the following steps (default FR_NORM_FULL).
+ * "flashrec 0.1.1 METADATA", §Features/Decoding: lm_head is evaluated only
+ * over the SID token range (FR_NORM_SID_RANGE: each live row streams only
+ * that range); "Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation step 4:
+ * probabilities over the candidate slice (FR_NORM_CANDIDATES: a beam's
+ * log-softmax runs over its allowed children, at temperature 1; no row is
+ * streamed).  Host-side setting; takes effect at the next fr_beam_step. */
+fr_status fr_beam_set_normalization(fr_beam* beam, fr_norm norm);
 
 /* Optional kernel timing.  While enabled, every fr_beam_step records CUDA
  * events around its two kernels on the step's stream.  fr_beam_read_timing

@@ -27,12 +27,13 @@ def torch_dtype(w: synth.Workload):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-def oracle_cfg(w: synth.Workload, B: Optional[int] = None, b_offset: int = 0, const: Optional[float] = None):
+def oracle_cfg(w: synth.Workload, B: Optional[int] = None, b_offset: int = 0, const: Optional[float] = None,
+               norm: int = 0):
     if const is not None:
-        cfg = oracle.Config.from_workload(w, mode=oracle.MODE_CONST, B=B, b_offset=b_offset)
+        cfg = oracle.Config.from_workload(w, mode=oracle.MODE_CONST, B=B, b_offset=b_offset, norm=norm)
         cfg.const_logit = const
         return cfg
-    return oracle.Config.from_workload(w, B=B, b_offset=b_offset)
+    return oracle.Config.from_workload(w, B=B, b_offset=b_offset, norm=norm)
 
 
 @dataclass
@@ -50,12 +51,14 @@ class GpuBeam:
     """A trie + beam on cuda:0, with the logits buffer and the generator."""
 
     def __init__(self, w: synth.Workload, sids: np.ndarray, b_offset: int = 0, ld: Optional[int] = None,
-                 misalign: int = 0):
+                 misalign: int = 0, norm: int = 0):
         self.w = w
         self.b_offset = b_offset
         self.sids_dev = torch.from_numpy(np.ascontiguousarray(sids, dtype=np.int32)).cuda()
         self.trie = fr.fr_trie_build(self.sids_dev, w.codebook_sizes, w.sid_base)
         self.beam = fr.fr_beam_init(self.trie, w.B, w.K, w.V, w.dtype)
+        if norm:
+            fr.fr_beam_set_normalization(self.beam, norm)
         self.ld = ld if ld is not None else w.V
         # `misalign` elements of offset make the row starts not 16-byte aligned
         n = w.B * w.K * self.ld + misalign

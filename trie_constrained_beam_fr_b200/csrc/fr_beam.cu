@@ -90,6 +90,8 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bm->shape.D = D;
     bm->shape.dtype = (int32_t)dtype;
     bm->shape.grid = sms;
+    bm->shape.norm = FR_NORM_FULL;
+    bm->shape.sid_span = (int32_t)(span - trie->sid_base);
     for (int t = 0; t < D; ++t) {
         // step t: live beams (1 at the root, then at most K) times the level's fan-out
         const int64_t bound = (int64_t)(t == 0 ? 1 : K) * std::max(1, trie->level_fanout[t]);
@@ -275,6 +277,13 @@ extern "C" fr_status fr_beam_set_state(fr_beam* bm, int32_t steps_done, const in
     bm->t = steps_done;
     bm->last_stream = s;
     return rc;
+}
+
+extern "C" fr_status fr_beam_set_normalization(fr_beam* bm, fr_norm norm) {
+    if (!bm || (norm != FR_NORM_FULL && norm != FR_NORM_SID_RANGE && norm != FR_NORM_CANDIDATES))
+        return FR_ERR_INVALID_ARG;
+    bm->shape.norm = (int32_t)norm;
+    return FR_OK;
 }
 
 extern "C" fr_status fr_beam_set_timing(fr_beam* bm, int32_t enable) {

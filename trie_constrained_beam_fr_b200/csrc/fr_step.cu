@@ -96,6 +96,8 @@ struct StreamArgs {
     const char* logits;
     int64_t ld;
     int32_t V, B, K, t, elt;
+    int64_t col0;  // each row's log-sum-exp runs over columns [col0, col0 + W)
+    int32_t W;
     const int32_t* live;
     const int32_t* node;
     const float* score;
@@ -110,8 +112,9 @@ struct StreamArgs {
 };
 
 struct Seg {
-    const char* ptr;     // row start
-    int64_t c0, c1;      // this CTA's element range in the row
+    const char* row;     // row start (the children's logits are gathered from it)
+    const char* ptr;     // start of the row's streamed window
+    int64_t c0, c1;      // this CTA's element range in the window
     int64_t a0, a1;      // 16-byte aligned interior of [c0, c1)
     int32_t b, k;
     int32_t nchunks;
@@ -174,12 +177,13 @@ __device__ __forceinline__ Seg make_seg(const StreamArgs& a, const int32_t* row_
     constexpr int64_t VE = 16 / ELT;          // elements per 16-byte vector
     constexpr int64_t CE = STAGE_BYTES / ELT;  // elements per chunk
     Seg g;
-    const int64_t rs = r * a.V;
+    const int64_t rs = r * a.W;
     g.c0 = max(bg, rs) - rs;
-    g.c1 = min(eg, rs + a.V) - rs;
+    g.c1 = min(eg, rs + a.W) - rs;
     g.b = find_request(row_start, a.B, r);
     g.k = (int32_t)(r - row_start[g.b]);
-    g.ptr = a.logits + ((int64_t)g.b * a.K + g.k) * a.ld * ELT;
+    g.row = a.logits + ((int64_t)g.b * a.K + g.k) * a.ld * ELT;
+    g.ptr = g.row + a.col0 * ELT;
     const uint32_t mis = (uint32_t)(reinterpret_cast<uint64_t>(g.ptr) + (uint64_t)(g.c0 * ELT)) & 15u;
     const int64_t pad = (int64_t)((16u - mis) & 15u) / ELT;
     g.a0 = min(g.c0 + pad, g.c1);
@@ -381,6 +385,16 @@ __device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f3
     }
 }
 
+// One element into a scalar (m, s): sum exp = exp(m) * s.
+__device__ __forceinline__ void lane_add_scalar(float& m, float& s, float x) {
+    if (x > m) {
+        s = s * ex2_approx((m - x) * L2E) + 1.0f;
+        m = x;
+    } else if (x != -INFINITY) {
+        s += ex2_approx((x - m) * L2E);  // a NaN lands here and poisons s
+    }
+}
+
 // One element (ragged head / tail of a segment) into (m, s2).
 __device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
     if (x > m) {
@@ -433,7 +447,7 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
             code[u] = i < nch ? __ldg(codes + i) : -1;
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.ptr, tb + code[u], a.elt) : 0.f;
+        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u], a.elt) : 0.f;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int32_t i = i0 + u * 32 + lane;
@@ -447,8 +461,8 @@ template <bool LSE_ONLY>
 __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
                                float s) {
     const int lane = threadIdx.x & 31;
-    const int64_t fc = (r * a.V) / Q;
-    const int64_t lc = ((r + 1) * a.V - 1) / Q;
+    const int64_t fc = (r * a.W) / Q;
+    const int64_t lc = ((r + 1) * a.W - 1) / Q;
     if (fc == lc) {
         finish_row<LSE_ONLY>(a, sg, m, s);
         return;
@@ -468,7 +482,7 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
         const int64_t gg = base + lane;
         float pm = -INFINITY, ps = 0.f;
         if (gg <= lc) {
-            const int sd = ((gg * Q) / a.V == r) ? 0 : 1;
+            const int sd = ((gg * Q) / a.W == r) ? 0 : 1;
             const float2 p = __ldcg(&a.partial[gg * 2 + sd]);
             pm = p.x;
             ps = p.y;
@@ -525,14 +539,14 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
     }
     __syncthreads();
 
-    const int64_t E = (int64_t)row_start[a.B] * a.V;
+    const int64_t E = (int64_t)row_start[a.B] * a.W;
     if (E == 0) return;
     const int64_t G = gridDim.x;
     const int64_t Q = ((E + G - 1) / G + GRAN - 1) / GRAN * GRAN;
     const int64_t bg = min(E, (int64_t)blockIdx.x * Q);
     const int64_t eg = min(E, (int64_t)(blockIdx.x + 1) * Q);
     if (bg >= eg) return;
-    const int64_t r_first = bg / a.V, r_last = (eg - 1) / a.V;
+    const int64_t r_first = bg / a.W, r_last = (eg - 1) / a.W;
 
     if (warp == PRODUCER_WARP) {
         if (lane == 0) {
@@ -673,6 +687,49 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
             m = -INFINITY;
             s2 = pack2(0.f, 0.f);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Candidate-slice normalisation ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation
+// step 4: probabilities over the candidate slice): a beam's log-softmax runs
+// over its allowed children only, so no logits row is streamed.  One warp per
+// live beam gathers the children's logits, takes their log-sum-exp and writes
+// the candidate scores s_k + (x - lse_slice).
+
+__global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    const int k = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int live = min(max(a.live[b], 0), a.K);
+    if (k >= live) return;
+    const int64_t bk = (int64_t)b * a.K + k;
+    const int t = a.t;
+    const int32_t n = a.node[bk];
+    if (n < 0 || n >= a.trie.nodes[t]) {
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const int32_t lo = a.trie.child_off[t][n], hi = a.trie.child_off[t][n + 1];
+    const int32_t base = a.cand_off[(int64_t)b * (a.K + 1) + k];
+    if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) {
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const char* row = a.logits + bk * a.ld * a.elt;
+    const int32_t* codes = a.trie.code[t + 1] + lo;
+    const int32_t tb = a.trie.tok_base[t];
+    const int32_t nch = hi - lo;
+    float m = -INFINITY, s = 0.f;
+    for (int32_t i = lane; i < nch; i += 32) lane_add_scalar(m, s, load_elem(row, tb + __ldg(codes + i), a.elt));
+    warp_combine(m, s);
+    const float lse = m + logf(s);
+    if (!isfinite(lse) && lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
+    const float sc = a.score[bk];
+    float* out = a.cand + (int64_t)b * a.cand_stride + base;
+    for (int32_t i = lane; i < nch; i += 32) {
+        const float x = load_elem(row, tb + __ldg(codes + i), a.elt);
+        out[i] = sc + (x - lse);
     }
 }
 
@@ -1218,6 +1275,8 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.K = sh.K;
     a.t = t;
     a.elt = sh.dtype == FR_BF16 ? 2 : 4;
+    a.col0 = sh.norm == FR_NORM_SID_RANGE ? trie.tok_base[0] : 0;
+    a.W = sh.norm == FR_NORM_SID_RANGE ? sh.sid_span : sh.V;
     a.live = cur.live;
     a.node = cur.node;
     a.score = cur.score;
@@ -1229,6 +1288,11 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.row_cnt = buf.row_cnt;
     a.err = buf.err;
     a.lse_out = nullptr;
+    if (sh.norm == FR_NORM_CANDIDATES) {
+        const dim3 grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
+        k_slice_candidates<<<grid, 256, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     const size_t smem = stream_smem_bytes(sh.B);
     if (sh.dtype == FR_BF16)
         k_stream<true, false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
@@ -1253,6 +1317,8 @@ cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_
     a.K = rows;
     a.t = 0;
     a.elt = dtype == FR_BF16 ? 2 : 4;
+    a.col0 = 0;
+    a.W = V;
     a.live = live_dev;
     a.partial = partial;
     a.row_cnt = row_cnt;

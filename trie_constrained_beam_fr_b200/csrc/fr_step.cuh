@@ -23,6 +23,8 @@ struct StepShape {
     int32_t B, K, V, D;
     int32_t dtype;  // fr_dtype
     int32_t grid;   // CTAs of the streaming kernel
+    int32_t norm;      // fr_norm: the set each row's log-softmax runs over
+    int32_t sid_span;  // C_0 + ... + C_{D-1}: width of the SID token range
     int32_t sel_cluster[FR_MAX_DEPTH];  // per step: CTAs per request of the cluster select (0: one CTA)
     int64_t sel_bound[FR_MAX_DEPTH];    // per step: most candidates a request can have
 };

@@ -33,6 +33,10 @@ FR_ERR_NOT_IN_CATALOG = 9
 FR_F32 = 0
 FR_BF16 = 1
 
+FR_NORM_FULL = 0
+FR_NORM_SID_RANGE = 1
+FR_NORM_CANDIDATES = 2
+
 # (name, restype, argtypes) of every function declared in include/fr.h
 _VP, _I32, _I64, _U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
 _P = ctypes.POINTER
@@ -53,6 +57,7 @@ FR_FUNCS = [
     ("fr_beam_status", _I32, [_VP]),
     ("fr_beam_get_state", _I32, [_VP, _P(_I32), _VP, _VP, _VP, _VP, _VP]),
     ("fr_beam_set_state", _I32, [_VP, _I32, _VP, _VP, _VP, _VP, _VP]),
+    ("fr_beam_set_normalization", _I32, [_VP, _I32]),
     ("fr_beam_set_timing", _I32, [_VP, _I32]),
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
@@ -258,6 +263,10 @@ def fr_beam_set_state(beam, steps_done: int, live: np.ndarray, prefix: np.ndarra
     return int(libfr().fr_beam_set_state(beam, int(steps_done), live.ctypes.data, prefix.ctypes.data,
                                          score.ctypes.data, None if kv is None else kv.ctypes.data,
                                          _stream(stream)))
+
+
+def fr_beam_set_normalization(beam, norm: int) -> None:
+    _check(libfr().fr_beam_set_normalization(beam, int(norm)), "fr_beam_set_normalization")
 
 
 def fr_beam_set_timing(beam, enable: bool) -> None:
