@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ref-requests", type=int, default=1, help="requests per reference-arm sample")
     p.add_argument("--batch", type=int, default=0, help="override B (requests per GPU), e.g. for profiling")
+    p.add_argument("--norm", default="full", choices=["full", "sid_range", "candidates"],
+                   help="log-softmax normalisation set (full vocabulary by default)")
     return p.parse_args()
 
 
@@ -281,6 +283,11 @@ def main():
     trie_ms = e0.elapsed_time(e1)
     levels = fr.fr_trie_level_sizes(trie)
     beam = fr.fr_beam_init(trie, B, K, V, w.dtype)
+    norm_code = {"full": fr.FR_NORM_FULL, "sid_range": fr.FR_NORM_SID_RANGE,
+                 "candidates": fr.FR_NORM_CANDIDATES}[args.norm]
+    fr.fr_beam_set_normalization(beam, norm_code)
+    # columns each live row's log-sum-exp streams (none over the candidate slice)
+    row_cols = {"full": V, "sid_range": w.depth * w.C, "candidates": 0}[args.norm]
 
     # one untimed decode produces every step's logits (prefix-dependent)
     bufs = [torch.empty((B, K, V), dtype=tdt, device=dev) for _ in range(D)]
@@ -298,7 +305,7 @@ def main():
     st = fr.fr_beam_status(beam)
     if st != fr.FR_OK:
         raise RuntimeError("decode failed: " + fr.fr_status_string(st))
-    bytes_per_decode = sum(r * V * elt for r in rows)
+    bytes_per_decode = sum(r * row_cols * elt for r in rows)
 
     def decode():
         fr.fr_beam_reset(beam)
@@ -334,13 +341,16 @@ def main():
     # roofline of the dominant kernel: the streaming log-sum-exp / candidate kernel
     peak, peak_kind = measured_peaks()
     n_launch = len(stream_ms)
-    per_step_bytes = [r * V * elt for r in rows]
+    per_step_bytes = [r * row_cols * elt for r in rows]
     alg_bytes = sum(per_step_bytes[i % D] for i in range(n_launch))
     stream_total_ms = float(np.sum(stream_ms))
     achieved = alg_bytes / (stream_total_ms / 1e3) / 1e9
     traffic = recorded_traffic(w.name)
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": traffic, "peak_source": peak_kind, "kernel": "k_stream",
+    if args.norm != "full":
+        traffic = None  # the committed counters are for the full-vocabulary stream
+    roofline = {"bound": "hbm" if row_cols else "latency", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                "kernel": "k_stream" if row_cols else "k_slice_candidates",
                 "alg_bytes_per_launch": alg_bytes / max(1, n_launch),
                 "ms_per_launch": stream_total_ms / max(1, n_launch)}
     per_step = []
@@ -349,7 +359,7 @@ def main():
         se = [select_ms[i] for i in range(t, n_launch, D)]
         per_step.append({"t": t, "live_rows": rows[t], "stream_us": 1e3 * float(np.mean(sm)),
                          "select_us": 1e3 * float(np.mean(se)),
-                         "stream_gbs": per_step_bytes[t] / (float(np.mean(sm)) / 1e3) / 1e9})
+                         "stream_gbs": per_step_bytes[t] / (float(np.mean(sm)) / 1e3) / 1e9 if sm else 0.0})
     hbm_gbs_decode = bytes_per_decode / (ms_per_decode / 1e3) / 1e9
 
     # end to end through the public API with host buffers
@@ -408,7 +418,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "B_per_gpu": B, "K": K, "depth": D, "V": V, "codes_per_level": w.C,
+            "config": {"workload": w.name, "norm": args.norm, "B_per_gpu": B, "K": K, "depth": D, "V": V,
+                       "codes_per_level": w.C,
                        "catalog": w.n_items, "logits": w.dtype, "trie_levels": levels,
                        "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"
                              % (B * K * V * elt / 1e9),

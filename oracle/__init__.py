@@ -54,7 +54,8 @@ class _Cfg(ctypes.Structure):
                 ("depth", ctypes.c_int32), ("sid_base", ctypes.c_int32),
                 ("codebook", ctypes.c_int32 * 16), ("mode", ctypes.c_int32),
                 ("const_logit", ctypes.c_float), ("seed", ctypes.c_uint64),
-                ("b_offset", ctypes.c_int64), ("norm", ctypes.c_int32)]
+                ("b_offset", ctypes.c_int64), ("norm", ctypes.c_int32),
+                ("temperature", ctypes.c_double), ("gseed", ctypes.c_uint64)]
 
 
 _lib = None
@@ -95,11 +96,13 @@ def lib():
         L.orc_step.restype = ctypes.c_int32
         L.orc_step.argtypes = [P(_Cfg), ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                P(ctypes.c_int32), P(ctypes.c_double), P(ctypes.c_int32), P(ctypes.c_double),
-                               P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double)]
+                               P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double), P(ctypes.c_double)]
         L.orc_decode.restype = ctypes.c_int
         L.orc_decode.argtypes = [P(_Cfg), ctypes.c_void_p, P(ctypes.c_int32), P(ctypes.c_double),
                                  P(ctypes.c_int64), P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double),
-                                 P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double)]
+                                 P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double), P(ctypes.c_double)]
+        L.orc_gumbel.restype = ctypes.c_double
+        L.orc_gumbel.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         L.orc_gen_seconds.restype = ctypes.c_double
         L.orc_gen_seconds.argtypes = [ctypes.c_int32]
     return _lib
@@ -125,6 +128,10 @@ def hash_logit(seed: int, b: int, prefix_h: int, v: int) -> float:
     return float(lib().orc_hash_logit(seed, b, prefix_h, v))
 
 
+def gumbel(gseed: int, b: int, t: int, k: int, token: int) -> float:
+    return float(lib().orc_gumbel(gseed & 0xFFFFFFFFFFFFFFFF, b, t, k, token))
+
+
 def round_bf16(x: float) -> float:
     return float(lib().orc_round_bf16(x))
 
@@ -144,6 +151,8 @@ class Config:
     seed: int = 0
     b_offset: int = 0
     norm: int = NORM_FULL
+    temperature: float = 0.0
+    gseed: int = 0
 
     @classmethod
     def from_workload(cls, w, mode: Optional[int] = None, B: Optional[int] = None,
@@ -156,7 +165,8 @@ class Config:
     def c(self) -> _Cfg:
         cb = (ctypes.c_int32 * 16)(*([int(x) for x in self.codebook] + [0] * (16 - len(self.codebook))))
         return _Cfg(self.B, self.K, self.V, self.depth, self.sid_base, cb, self.mode,
-                    self.const_logit, self.seed & 0xFFFFFFFFFFFFFFFF, self.b_offset, self.norm)
+                    self.const_logit, self.seed & 0xFFFFFFFFFFFFFFFF, self.b_offset, self.norm,
+                    float(self.temperature), self.gseed & 0xFFFFFFFFFFFFFFFF)
 
     def token_base(self, level: int) -> int:
         return self.sid_base + int(sum(self.codebook[:level]))
@@ -228,7 +238,8 @@ class StepResult:
     score: np.ndarray    # [K] float64
     parent: np.ndarray   # [K]
     token: np.ndarray    # [K]
-    excluded_best: float  # best candidate score that did not survive (-inf if none)
+    excluded_best: float  # key of the best candidate that did not survive (-inf if none)
+    key: np.ndarray = None  # [K] keys the survivors were ranked by
 
 
 def step(cfg: Config, cat: Catalog, b: int, t: int, live: int, prefix: np.ndarray,
@@ -242,13 +253,14 @@ def step(cfg: Config, cat: Catalog, b: int, t: int, live: int, prefix: np.ndarra
     par = np.empty(K, dtype=np.int32)
     tok = np.empty(K, dtype=np.int32)
     exc = ctypes.c_double()
+    key = np.empty(K, dtype=np.float64)
     c = cfg.c()
     nl = lib().orc_step(ctypes.byref(c), cat.handle, b, t, live, _ptr(pre, ctypes.c_int32), _ptr(sc, ctypes.c_double),
                         _ptr(npre, ctypes.c_int32), _ptr(nsc, ctypes.c_double), _ptr(par, ctypes.c_int32),
-                        _ptr(tok, ctypes.c_int32), ctypes.byref(exc))
+                        _ptr(tok, ctypes.c_int32), ctypes.byref(exc), _ptr(key, ctypes.c_double))
     if nl < 0:
         raise ValueError("oracle step rejected its arguments")
-    return StepResult(int(nl), npre, nsc, par, tok, float(exc.value))
+    return StepResult(int(nl), npre, nsc, par, tok, float(exc.value), key)
 
 
 @dataclass
@@ -261,7 +273,8 @@ class DecodeResult:
     step_score: np.ndarray    # [D, B, K]
     step_live: np.ndarray     # [D, B]
     step_prefix: np.ndarray   # [D, B, K, D]
-    step_excluded: np.ndarray  # [D, B] best non-surviving candidate score (-inf if none)
+    step_excluded: np.ndarray  # [D, B] key of the best non-surviving candidate (-inf if none)
+    step_key: np.ndarray       # [D, B, K] keys the survivors were ranked by (= scores at temperature 0)
     gen_seconds: float = 0.0
 
 
@@ -276,13 +289,14 @@ def decode(cfg: Config, cat: Catalog) -> DecodeResult:
     sl = np.empty((D, B), dtype=np.int32)
     spre = np.empty((D, B, K, D), dtype=np.int32)
     sexc = np.empty((D, B), dtype=np.float64)
+    skey = np.empty((D, B, K), dtype=np.float64)
     c = cfg.c()
     lib().orc_gen_seconds(1)
     rc = lib().orc_decode(ctypes.byref(c), cat.handle, _ptr(sids, ctypes.c_int32), _ptr(scores, ctypes.c_double),
                           _ptr(items, ctypes.c_int64), _ptr(sp, ctypes.c_int32), _ptr(st, ctypes.c_int32),
                           _ptr(ss, ctypes.c_double), _ptr(sl, ctypes.c_int32), _ptr(spre, ctypes.c_int32),
-                          _ptr(sexc, ctypes.c_double))
+                          _ptr(sexc, ctypes.c_double), _ptr(skey, ctypes.c_double))
     if rc != 0:
         raise ValueError("oracle decode failed: %s" % ERR_NAMES.get(rc, rc))
     gen = float(lib().orc_gen_seconds(1))
-    return DecodeResult(sids, scores, items, sp, st, ss, sl, spre, sexc, gen)
+    return DecodeResult(sids, scores, items, sp, st, ss, sl, spre, sexc, skey, gen)

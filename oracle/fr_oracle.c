@@ -27,8 +27,14 @@
  *  - normalisation over the full vocabulary V (not the SID range);
  *  - a request starts from one live root beam (empty prefix, score 0), the
  *    other K-1 slots dead;
- *  - total order: score descending, then parent slot ascending, then token
- *    ascending;
+ *  - total order: key descending, then parent slot ascending, then token
+ *    ascending; the key is the running score at temperature 0;
+ *  - temperature T > 0 ("flashrec 0.1.1 METADATA", §Serving/API: Gumbel
+ *    top-k without replacement above temperature 0): each step ranks a
+ *    candidate by key = score / T + G with G an independent Gumbel(0, 1)
+ *    draw per (request, step, parent slot, token) from a counter-based
+ *    SplitMix64 stream (orc_gumbel); survivors keep their unperturbed score
+ *    (the sum of log-probabilities) and are emitted in key order;
  *  - fewer than K candidates leaves the remaining slots dead;
  *  - duplicate catalog rows: the first row is kept (dedupe) or the catalog is
  *    rejected; a code outside [0, C_l) rejects the catalog;
@@ -110,6 +116,21 @@ float orc_round_bf16(float x) {
     return r;
 }
 
+/* Gumbel(0, 1) noise of candidate (request b, step t, parent slot k, token):
+ * U = ((u >> 40) + 1/2) * 2^-24 in (0, 1) from the counter-based draw
+ * u = splitmix64(splitmix64(splitmix64(splitmix64(gseed) ^ b) ^ t) ^ (k * 2^32 + token)),
+ * G = -log(-log U).  Adding G to log-weights and keeping the top K samples K
+ * items without replacement from the softmax of the log-weights (the
+ * Gumbel-top-k trick). */
+double orc_gumbel(uint64_t gseed, int64_t b, int32_t t, int32_t k, int32_t token) {
+    uint64_t h = orc_splitmix64(gseed);
+    h = orc_splitmix64(h ^ (uint64_t)b);
+    h = orc_splitmix64(h ^ (uint64_t)(uint32_t)t);
+    uint64_t u = orc_splitmix64(h ^ ((uint64_t)(uint32_t)k << 32 | (uint64_t)(uint32_t)token));
+    double U = ((double)(u >> 40) + 0.5) * 0x1p-24;
+    return -log(-log(U));
+}
+
 /* ------------------------------------------------------------------------- */
 /* Workload description.                                                      */
 
@@ -122,6 +143,8 @@ typedef struct {
     uint64_t seed;
     int64_t b_offset;   /* request index of local request 0 in the hash */
     int32_t norm;       /* ORC_NORM_*: the set the log-softmax normalises over */
+    double temperature; /* 0: deterministic top-K; > 0: Gumbel top-K */
+    uint64_t gseed;     /* seed of the Gumbel noise */
 } orc_cfg;
 
 static int32_t level_token_base(const orc_cfg* cfg, int32_t level) {
@@ -301,18 +324,20 @@ int64_t orc_find_row(const orc_catalog* c, const int32_t* sid) {
 /* One beam-search step for one request.                                      */
 
 typedef struct {
-    double score;
+    double key;    /* what the selection ranks: the score, or its Gumbel-perturbed form */
+    double score;  /* running score: sum of log-probabilities */
     int32_t parent;
     int32_t token;
     int32_t code;
 } orc_cand;
 
-/* Strict total order: higher score first, then lower parent slot, then lower
- * token (the lowest flat (parent, token) index wins a tie). */
+/* Strict total order: higher key first (the score, or at temperature > 0 the
+ * Gumbel-perturbed score), then lower parent slot, then lower token (the
+ * lowest flat (parent, token) index wins a tie). */
 static int cmp_cand(const void* pa, const void* pb) {
     const orc_cand* a = (const orc_cand*)pa;
     const orc_cand* b = (const orc_cand*)pb;
-    if (a->score != b->score) return a->score > b->score ? -1 : 1;
+    if (a->key != b->key) return a->key > b->key ? -1 : 1;
     if (a->parent != b->parent) return a->parent < b->parent ? -1 : 1;
     return (a->token > b->token) - (a->token < b->token);
 }
@@ -330,12 +355,14 @@ static double now_seconds(void) {
  *   score:       [K] running score of each live beam
  * Outputs (all [K], slots >= new live are dead: parent/token/code -1, score -inf):
  *   new_prefix   [K, depth], new_score [K], parent [K], token [K]
- *   excluded_best  (may be NULL) score of the best candidate that did not
+ *   excluded_best  (may be NULL) key of the best candidate that did not
  *                  survive, -inf if every candidate survived
+ *   new_key        (may be NULL) [K] key each survivor was ranked by (its score
+ *                  at temperature 0), -inf for dead slots
  * Returns the new live count, or -1 on error. */
 int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t t, int32_t live,
                  const int32_t* prefix, const double* score, int32_t* new_prefix, double* new_score,
-                 int32_t* parent, int32_t* token, double* excluded_best) {
+                 int32_t* parent, int32_t* token, double* excluded_best, double* new_key) {
     const int32_t K = cfg->K, D = cfg->depth;
     if (t < 0 || t >= D || live < 0 || live > K) return -1;
     float* row = (float*)malloc(sizeof(float) * (size_t)cfg->V);
@@ -366,6 +393,9 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
         for (int32_t i = 0; i < nk; ++i) {
             int32_t tok = tok_base + kids[i];
             cand[nc].score = score[k] + ((double)row[tok] - lse);
+            cand[nc].key = (cfg->temperature > 0.0)
+                               ? cand[nc].score / cfg->temperature + orc_gumbel(cfg->gseed, b + cfg->b_offset, t, k, tok)
+                               : cand[nc].score;
             cand[nc].parent = k;
             cand[nc].token = tok;
             cand[nc].code = kids[i];
@@ -374,18 +404,20 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     }
     qsort(cand, (size_t)nc, sizeof(orc_cand), cmp_cand);
     int32_t nlive = (int32_t)(nc < K ? nc : K);
-    if (excluded_best) *excluded_best = (nc > nlive) ? cand[nlive].score : -INFINITY;
+    if (excluded_best) *excluded_best = (nc > nlive) ? cand[nlive].key : -INFINITY;
     for (int32_t j = 0; j < K; ++j) {
         if (j < nlive) {
             const orc_cand* c = &cand[j];
             for (int32_t l = 0; l < D; ++l) new_prefix[j * D + l] = (l < t) ? prefix[c->parent * D + l] : -1;
             new_prefix[j * D + t] = c->code;
             new_score[j] = c->score;
+            if (new_key) new_key[j] = c->key;
             parent[j] = c->parent;
             token[j] = c->token;
         } else {
             for (int32_t l = 0; l < D; ++l) new_prefix[j * D + l] = -1;
             new_score[j] = -INFINITY;
+            if (new_key) new_key[j] = -INFINITY;
             parent[j] = -1;
             token[j] = -1;
         }
@@ -404,12 +436,14 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
  *   items  [B, K] catalog row of each final SID (-1 dead),
  *   step_parent / step_token [depth, B, K], step_score [depth, B, K],
  *   step_live [depth, B]   (state after each step),
- *   step_prefix [depth, B, K, depth] and step_excluded [depth, B] (optional).
+ *   step_prefix [depth, B, K, depth], step_excluded [depth, B] and the keys
+ *   the survivors were ranked by, step_key [depth, B, K] (optional).
  * Returns ORC_OK or an error. */
 int orc_decode(const orc_cfg* cfg, const orc_catalog* cat, int32_t* sids, double* scores, int64_t* items,
                int32_t* step_parent, int32_t* step_token, double* step_score, int32_t* step_live,
                int32_t* step_prefix /* [depth, B, K, depth] or NULL */,
-               double* step_excluded /* [depth, B] or NULL */) {
+               double* step_excluded /* [depth, B] or NULL */,
+               double* step_key /* [depth, B, K] or NULL */) {
     const int32_t B = cfg->B, K = cfg->K, D = cfg->depth;
     int32_t* pre = (int32_t*)malloc(sizeof(int32_t) * (size_t)K * D);
     int32_t* npre = (int32_t*)malloc(sizeof(int32_t) * (size_t)K * D);
@@ -425,7 +459,8 @@ int orc_decode(const orc_cfg* cfg, const orc_catalog* cat, int32_t* sids, double
             int32_t* par = step_parent + ((int64_t)t * B + b) * K;
             int32_t* tok = step_token + ((int64_t)t * B + b) * K;
             live = orc_step(cfg, cat, b, t, live, pre, sc, npre, nsc, par, tok,
-                            step_excluded ? step_excluded + (int64_t)t * B + b : NULL);
+                            step_excluded ? step_excluded + (int64_t)t * B + b : NULL,
+                            step_key ? step_key + ((int64_t)t * B + b) * K : NULL);
             if (live < 0) {
                 free(pre); free(npre); free(sc); free(nsc);
                 return ORC_ERR_ARG;

@@ -24,8 +24,18 @@ MUTANTS = {
     "subset_lse_drops_max": ("for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);\n    return m + log(s);",
                              "for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);\n    return log(s);"),
     "lse_max_wrong_way": ("if ((double)x[v] > m) m = (double)x[v];", "if ((double)x[v] < m) m = (double)x[v];"),
-    "order_ascending": ("if (a->score != b->score) return a->score > b->score ? -1 : 1;",
-                        "if (a->score != b->score) return a->score < b->score ? -1 : 1;"),
+    "order_ascending": ("if (a->key != b->key) return a->key > b->key ? -1 : 1;",
+                        "if (a->key != b->key) return a->key < b->key ? -1 : 1;"),
+    "ranks_by_score_not_key": ("if (a->key != b->key) return a->key > b->key ? -1 : 1;",
+                               "if (a->score != b->score) return a->score > b->score ? -1 : 1;"),
+    "gumbel_sign": ("return -log(-log(U));", "return log(-log(U));"),
+    "temperature_multiplies": ("? cand[nc].score / cfg->temperature + orc_gumbel(",
+                               "? cand[nc].score * cfg->temperature + orc_gumbel("),
+    "gumbel_counter_drops_step": ("h = orc_splitmix64(h ^ (uint64_t)(uint32_t)t);", "h = orc_splitmix64(h);"),
+    "gumbel_counter_drops_slot": ("((uint64_t)(uint32_t)k << 32 | (uint64_t)(uint32_t)token)",
+                                  "((uint64_t)(uint32_t)token)"),
+    "noise_in_kept_score": ("new_score[j] = c->score;\n            if (new_key)",
+                            "new_score[j] = c->key;\n            if (new_key)"),
     "tie_parent_reversed": ("if (a->parent != b->parent) return a->parent < b->parent ? -1 : 1;",
                             "if (a->parent != b->parent) return a->parent > b->parent ? -1 : 1;"),
     "tie_token_reversed": ("return (a->token > b->token) - (a->token < b->token);",

@@ -356,3 +356,134 @@ def test_greedy_path_does_not_depend_on_the_normalisation():
         cfg.norm = norm
         paths.append(oracle.decode(cfg, cat).sids[0, 0].tolist())
     assert paths[0] == paths[1] == paths[2]
+
+
+# --------------------------------------------------------------------------
+# Sampling at temperature > 0 (Gumbel top-K): "flashrec 0.1.1 METADATA",
+# §Features, lists temperature sampling beside the deterministic beam.  Adding
+# independent Gumbel(0, 1) noise to log-weights / T and keeping the K largest
+# draws K items without replacement with Plackett-Luce probabilities of
+# softmax(log-weights / T) (the Gumbel-max theorem and its top-K extension).
+
+EULER_GAMMA = 0.5772156649015329
+
+
+def test_gumbel_noise_is_standard_gumbel_and_distinct_per_counter():
+    from scipy import stats
+    # U has 24 random bits, so a grid of ~2000 counters is collision-free with
+    # high probability while a counter that ignores one field repeats values
+    small = np.array([oracle.gumbel(7, b, t, k, tok) for b in range(4) for t in range(4) for k in range(8)
+                      for tok in range(16)])
+    assert len(np.unique(small)) == small.size, "noise repeats across (request, step, slot, token)"
+    g = np.array([oracle.gumbel(7, b, t, k, tok) for b in range(25) for t in range(4) for k in range(20)
+                  for tok in range(20)])
+    n = g.size
+    assert abs(g.mean() - EULER_GAMMA) < 5 * math.pi / math.sqrt(6 * n)
+    assert g.var() == pytest.approx(math.pi ** 2 / 6, rel=0.03)
+    assert stats.kstest(g, stats.gumbel_r.cdf).pvalue > 1e-4
+    # another seed gives other noise
+    assert oracle.gumbel(8, 0, 0, 0, 0) != oracle.gumbel(7, 0, 0, 0, 0)
+
+
+def _one_level(B, K, T, gseed=11, mode=oracle.MODE_HASH_F32):
+    """B requests over a one-level catalog of all 16 codes; per request the
+    exact sampling probabilities softmax(logit / T) over the 16 SID tokens."""
+    w, sids, cfg = _tiny_cfg(K, 16, mode, seed=2, V=64, C=16, D=1, sid_base=30)
+    cfg.B = B
+    cfg.temperature = T
+    cfg.gseed = gseed
+    res = oracle.decode(cfg, oracle.Catalog(sids, w.codebook_sizes))
+    probs = np.empty((B, 16))
+    for b in range(B):
+        r = oracle.fill_row(cfg, b, []).astype(np.float64)[30:46] / T
+        probs[b] = np.exp(r - logsumexp(r))
+    return res, probs
+
+
+def _chi2_pvalue(observed, expected):
+    from scipy import stats
+    keep = expected >= 5
+    o = np.append(observed[keep], observed[~keep].sum())
+    e = np.append(expected[keep], expected[~keep].sum())
+    if e[-1] < 5:
+        o, e = o[:-1], e[:-1]
+    return stats.chi2.sf(((o - e) ** 2 / e).sum(), len(o) - 1)
+
+
+@pytest.mark.parametrize("T", [0.7, 1.5])
+def test_gumbel_max_samples_the_tempered_softmax(T):
+    """K = 1: the one survivor is a draw from softmax(log-prob / T).  The
+    request's candidates are binned by their probability rank; the count of
+    draws in each bin must match the sum of the exact probabilities."""
+    B = 20000
+    res, probs = _one_level(B, 1, T)
+    order = np.argsort(-probs, axis=1, kind="stable")
+    rank_of = np.argsort(order, axis=1)
+    chosen = res.sids[:, 0, 0]
+    observed = np.bincount(rank_of[np.arange(B), chosen], minlength=16).astype(float)
+    expected = np.take_along_axis(probs, order, axis=1).sum(axis=0)
+    assert _chi2_pvalue(observed, expected) > 1e-4
+
+
+def test_gumbel_top2_is_plackett_luce():
+    """K = 2: the ordered pair (first, second) has probability
+    p_i * p_j / (1 - p_i) -- sampling without replacement."""
+    B, T = 30000, 1.0
+    res, probs = _one_level(B, 2, T, gseed=3)
+    order = np.argsort(-probs, axis=1, kind="stable")
+    rank_of = np.argsort(order, axis=1)
+    a = rank_of[np.arange(B), res.sids[:, 0, 0]]
+    c = rank_of[np.arange(B), res.sids[:, 1, 0]]
+    assert np.all(a != c)
+    R = 4
+    observed = np.zeros(R * R + 1)
+    expected = np.zeros(R * R + 1)
+    ps = np.take_along_axis(probs, order, axis=1)
+    for i in range(R):
+        for j in range(R):
+            if i == j:
+                continue
+            observed[i * R + j] = np.count_nonzero((a == i) & (c == j))
+            expected[i * R + j] = (ps[:, i] * ps[:, j] / (1 - ps[:, i])).sum()
+    observed[-1] = B - observed[:-1].sum()
+    expected[-1] = B - expected[:-1].sum()
+    assert _chi2_pvalue(observed, expected) > 1e-4
+
+
+def test_gumbel_scores_are_unperturbed_and_keys_ordered():
+    """With K at least the catalog size every SID survives whatever the noise;
+    the kept scores are the brute-force log-probabilities of their SIDs, and
+    the survivors are ordered by non-increasing key."""
+    for T in (0.3, 1.0, 4.0):
+        w, sids, cfg = _tiny_cfg(600, 500, oracle.MODE_HASH_BF16, seed=4, catalog_seed=4)
+        cfg.temperature = T
+        cfg.gseed = 99
+        res = oracle.decode(cfg, oracle.Catalog(sids, w.codebook_sizes))
+        bf = {sid: s for s, sid in _brute_force(cfg, sids)}
+        n = len(bf)
+        assert res.step_live[-1, 0] == n
+        got = {tuple(x): s for x, s in zip(res.sids[0, :n].tolist(), res.scores[0, :n])}
+        assert set(got) == set(bf)
+        for sid, s in got.items():
+            assert s == pytest.approx(bf[sid], abs=1e-9)
+        for t in range(cfg.depth):
+            k = res.step_key[t, 0, : res.step_live[t, 0]]
+            assert np.all(k[:-1] >= k[1:])
+        # the noise reorders the beam (it is not ranked by score any more)
+        assert np.any(np.diff(res.scores[0, :n]) > 0)
+
+
+def test_gumbel_vanishing_temperature_is_the_deterministic_beam():
+    """As T -> 0 the key is dominated by score / T, so the sampled beam is the
+    deterministic top-K wherever the scores are not within noise * T."""
+    w, sids, cfg = _tiny_cfg(8, 500, oracle.MODE_HASH_F32, seed=1, catalog_seed=1)
+    cfg.B = 6
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    det = oracle.decode(cfg, cat)
+    cfg.temperature = 1e-12
+    cfg.gseed = 5
+    cold = oracle.decode(cfg, cat)
+    np.testing.assert_array_equal(cold.sids, det.sids)
+    np.testing.assert_allclose(cold.scores, det.scores, atol=0)
+    cfg.temperature = 0.0
+    assert np.array_equal(oracle.decode(cfg, cat).step_key, det.step_score)
