@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--batch", type=int, default=0, help="override B (requests per GPU), e.g. for profiling")
     p.add_argument("--norm", default="full", choices=["full", "sid_range", "candidates"],
                    help="log-softmax normalisation set (full vocabulary by default)")
+    p.add_argument("--temperature", type=float, default=0.0,
+                   help="0: deterministic top-K; > 0: Gumbel top-K sampling at this temperature")
     return p.parse_args()
 
 
@@ -185,14 +187,20 @@ class ClockSampler:
 # CPU oracle timing (reference arm and cpu_baseline)
 
 
-def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, sids=None, cat=None):
+NORM_CODES = {"full": 0, "sid_range": 1, "candidates": 2}  # fr_norm values (include/fr.h)
+
+
+def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, sids=None, cat=None,
+                  norm: str = "full", temperature: float = 0.0):
     import oracle
 
     if sids is None:
         sids = synth.workload_catalog(w)
     if cat is None:
         cat = oracle.Catalog(sids, w.codebook_sizes)
-    cfg = oracle.Config.from_workload(w, B=n_requests, b_offset=first_request)
+    cfg = oracle.Config.from_workload(w, B=n_requests, b_offset=first_request, norm=NORM_CODES[norm])
+    cfg.temperature = temperature
+    cfg.gseed = 0x5EED
     t0 = time.perf_counter()
     r = oracle.decode(cfg, cat)
     wall = time.perf_counter() - t0
@@ -210,8 +218,10 @@ def run_reference(args):
     sids = synth.workload_catalog(w)
     cat = oracle.Catalog(sids, w.codebook_sizes)
     for i in range(args.warmup):
-        oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat)
-    samples = [oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat)
+        oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
+                      temperature=args.temperature)
+    samples = [oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
+                             temperature=args.temperature)
                for i in range(args.steps)]
     cand = sum(s["candidates"] for s in samples)
     secs = sum(s["method_s"] for s in samples)
@@ -222,7 +232,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "K": w.K, "depth": w.depth, "V": w.V, "codes_per_level": w.C,
+        "config": {"workload": w.name, "norm": args.norm, "temperature": args.temperature, "B": w.B, "K": w.K, "depth": w.depth, "V": w.V, "codes_per_level": w.C,
                    "catalog": w.n_items, "logits": w.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -286,6 +296,8 @@ def main():
     norm_code = {"full": fr.FR_NORM_FULL, "sid_range": fr.FR_NORM_SID_RANGE,
                  "candidates": fr.FR_NORM_CANDIDATES}[args.norm]
     fr.fr_beam_set_normalization(beam, norm_code)
+    if args.temperature > 0:
+        fr.fr_beam_set_sampling(beam, args.temperature, 0x5EED, b_offset)
     # columns each live row's log-sum-exp streams (none over the candidate slice)
     row_cols = {"full": V, "sid_range": w.depth * w.C, "candidates": 0}[args.norm]
 
@@ -406,7 +418,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s = oracle_sample(w, 1, first_request=0, sids=sids_np)
+        s = oracle_sample(w, 1, first_request=0, sids=sids_np, norm=args.norm, temperature=args.temperature)
         cpu = {"value": s["candidates"] / s["method_s"], "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "request 0 of %s (1 of B=%d), full decode, single-threaded C oracle in double, "
                          "time excluding its logits generation (%.1f s method, %.1f s generation)"
@@ -418,7 +430,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "norm": args.norm, "B_per_gpu": B, "K": K, "depth": D, "V": V,
+            "config": {"workload": w.name, "norm": args.norm, "temperature": args.temperature, "B_per_gpu": B, "K": K, "depth": D, "V": V,
                        "codes_per_level": w.C,
                        "catalog": w.n_items, "logits": w.dtype, "trie_levels": levels,
                        "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"

@@ -193,6 +193,21 @@ fr_status fr_beam_set_state(fr_beam* beam, int32_t steps_done, const int32_t* li
  * streamed).  Host-side setting; takes effect at the next fr_beam_step. */
 fr_status fr_beam_set_normalization(fr_beam* beam, fr_norm norm);
 
+/* Sampling of the following steps ("flashrec 0.1.1 METADATA", §Serving/API:
+ * deterministic top-k at temperature 0, Gumbel top-k without replacement
+ * above it).  temperature == 0 (the default) keeps the deterministic top-K.
+ * temperature > 0 ranks each candidate by key = score / temperature + G,
+ * where G = -log(-log U) and U = ((u >> 40) + 1/2) * 2^-24, with
+ *   u = splitmix64(splitmix64(splitmix64(splitmix64(seed) ^ b') ^ t) ^ (k * 2^32 + token)),
+ * b' = request_offset + b (the request's index in the stream), t the step,
+ * k the parent slot and token the candidate's vocabulary id.  The K
+ * largest keys survive (ties: lowest (parent slot, token)); survivors are
+ * emitted in key order and keep their unperturbed score (the sum of
+ * log-probabilities).  Returns FR_ERR_INVALID_ARG for a negative, NaN or
+ * infinite temperature, one whose reciprocal overflows, or a negative
+ * request_offset.  Host-side setting; takes effect at the next fr_beam_step. */
+fr_status fr_beam_set_sampling(fr_beam* beam, float temperature, uint64_t seed, int64_t request_offset);
+
 /* Optional kernel timing.  While enabled, every fr_beam_step records CUDA
  * events around its two kernels on the step's stream.  fr_beam_read_timing
  * synchronises, returns up to max_steps per-step durations in milliseconds

@@ -6,6 +6,7 @@
 // for the contract of each call.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <math.h>
 #include <string.h>
 
 #include <algorithm>
@@ -110,7 +111,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
         bytes += align256(sizeof(int32_t) * (size_t)B);            // live
     }
     bytes += 2 * align256(sizeof(int32_t) * bk);                   // parent, token
-    bytes += align256(sizeof(float) * (size_t)B * cand_stride);    // cand
+    bytes += 2 * align256(sizeof(float) * (size_t)B * cand_stride);  // cand, cand_key
     bytes += align256(sizeof(float2) * (size_t)sms * 2);           // partial
     bytes += align256(sizeof(int32_t) * bk);                       // row_cnt
     bytes += align256(sizeof(int32_t));                            // err
@@ -134,6 +135,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bm->buf.parent = carve<int32_t>(p, bk);
     bm->buf.token = carve<int32_t>(p, bk);
     bm->buf.cand = carve<float>(p, (size_t)B * cand_stride);
+    bm->buf.cand_key = carve<float>(p, (size_t)B * cand_stride);
     bm->buf.cand_stride = cand_stride;
     bm->buf.partial = carve<float2>(p, (size_t)sms * 2);
     bm->buf.row_cnt = carve<int32_t>(p, bk);
@@ -283,6 +285,19 @@ extern "C" fr_status fr_beam_set_normalization(fr_beam* bm, fr_norm norm) {
     if (!bm || (norm != FR_NORM_FULL && norm != FR_NORM_SID_RANGE && norm != FR_NORM_CANDIDATES))
         return FR_ERR_INVALID_ARG;
     bm->shape.norm = (int32_t)norm;
+    return FR_OK;
+}
+
+extern "C" fr_status fr_beam_set_sampling(fr_beam* bm, float temperature, uint64_t seed, int64_t request_offset) {
+    if (!bm || !(temperature >= 0.f) || !isfinite(temperature) || request_offset < 0) return FR_ERR_INVALID_ARG;
+    float inv = 0.f;
+    if (temperature > 0.f) {
+        inv = 1.0f / temperature;
+        if (!isfinite(inv)) return FR_ERR_INVALID_ARG;
+    }
+    bm->shape.inv_temp = inv;
+    bm->shape.gseed = seed;
+    bm->shape.req_offset = request_offset;
     return FR_OK;
 }
 

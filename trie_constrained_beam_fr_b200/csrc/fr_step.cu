@@ -28,6 +28,12 @@
 //            reorder gathers: backpointer, token, trie node, score, prefix and
 //            KV slot of every survivor, and the next step's candidate offsets.
 //
+// Above temperature 0 ("flashrec 0.1.1 METADATA", §Serving/API: Gumbel top-k
+// without replacement) the candidate writers also store a perturbed key
+// score / T + G per candidate, G a Gumbel(0, 1) draw from a counter-based
+// SplitMix64 stream indexed by (request, step, parent slot, token); k_select
+// ranks the keys and the survivors keep their unperturbed scores.
+//
 // Every wait on an mbarrier is bounded: after 2 s the kernel records
 // FR_ERR_DEVICE in the beam's status word and returns.
 #include <cooperative_groups.h>
@@ -109,7 +115,38 @@ struct StreamArgs {
     int32_t* row_cnt;
     int32_t* err;
     float* lse_out;  // log-sum-exp-only instantiation: lse of row (0, k) at lse_out[k]
+    float* cand_key;     // sampling: perturbed keys beside cand (null at temperature 0)
+    float inv_temp;      // 1 / temperature
+    uint64_t gseed;      // seed of the Gumbel stream
+    int64_t req_offset;  // index of local request 0 in the Gumbel stream
 };
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the finaliser of a Weyl
+// sequence, used here as a counter-based generator.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+    uint64_t z = x + 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// The part of the Gumbel counter shared by a row's candidates: request and step.
+__device__ __forceinline__ uint64_t gumbel_row_hash(uint64_t gseed, int64_t b, int t) {
+    return splitmix64(splitmix64(splitmix64(gseed) ^ (uint64_t)b) ^ (uint64_t)(uint32_t)t);
+}
+
+// Gumbel(0, 1) draw of candidate (parent slot k, token) of a row:
+// G = -log(-log U), U = (m + 1/2) * 2^-24, m the top 24 bits of the draw.
+// U itself is not a float for m >= 2^23 (25 significant bits), so -log U is
+// taken from the exact float U = (2m + 1) * 2^-25 when m < 2^23 and from the
+// exact float 1 - U = (2^25 - 2m - 1) * 2^-25 through log1p otherwise.
+__device__ __forceinline__ float gumbel_noise(uint64_t row_hash, int32_t k, int32_t token) {
+    const uint64_t u = splitmix64(row_hash ^ (((uint64_t)(uint32_t)k << 32) | (uint64_t)(uint32_t)token));
+    const uint32_t m = (uint32_t)(u >> 40);
+    const float e = (m < (1u << 23)) ? -logf((float)(2u * m + 1u) * 0x1p-25f)
+                                     : -log1pf(-(float)((1u << 25) - 2u * m - 1u) * 0x1p-25f);
+    return -logf(e);
+}
 
 struct Seg {
     const char* row;     // row start (the children's logits are gathered from it)
@@ -437,6 +474,17 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
     const int32_t tb = a.trie.tok_base[t];
     float* out = a.cand + (int64_t)sg.b * a.cand_stride + base;
     const int32_t nch = hi - lo;
+    if (a.cand_key) {
+        float* key = a.cand_key + (int64_t)sg.b * a.cand_stride + base;
+        const uint64_t rh = gumbel_row_hash(a.gseed, a.req_offset + sg.b, t);
+        for (int32_t i = lane; i < nch; i += 32) {
+            const int32_t tok = tb + __ldg(codes + i);
+            const float v = sc + (load_elem(sg.row, tok, a.elt) - lse);
+            out[i] = v;
+            key[i] = v * a.inv_temp + gumbel_noise(rh, sg.k, tok);
+        }
+        return;
+    }
     constexpr int U = 8;  // independent gathers in flight per lane
     for (int32_t i0 = 0; i0 < nch; i0 += 32 * U) {
         int32_t code[U];
@@ -727,9 +775,13 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
     if (!isfinite(lse) && lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
     const float sc = a.score[bk];
     float* out = a.cand + (int64_t)b * a.cand_stride + base;
+    float* key = a.cand_key ? a.cand_key + (int64_t)b * a.cand_stride + base : nullptr;
+    const uint64_t rh = key ? gumbel_row_hash(a.gseed, a.req_offset + b, t) : 0ull;
     for (int32_t i = lane; i < nch; i += 32) {
-        const float x = load_elem(row, tb + __ldg(codes + i), a.elt);
-        out[i] = sc + (x - lse);
+        const int32_t tok = tb + __ldg(codes + i);
+        const float v = sc + (load_elem(row, tok, a.elt) - lse);
+        out[i] = v;
+        if (key) key[i] = v * a.inv_temp + gumbel_noise(rh, k, tok);
     }
 }
 
@@ -746,7 +798,8 @@ struct SelectArgs {
     StateDev cur, nxt;
     TrieDev trie;
     int32_t B, K, D, t;
-    const float* cand;
+    const float* cand;  // candidate scores (what survivors keep)
+    const float* rank;  // what the selection ranks: cand, or the perturbed keys
     int64_t cand_stride;
     int32_t* parent_out;
     int32_t* token_out;
@@ -790,7 +843,7 @@ __device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, 
     if (j == 0) cand_off_row[K] = tot;
 }
 
-// Sorts the Kp winners in sel (descending (key, ~slot), so score descending,
+// Sorts the Kp winners in sel (descending (key, ~slot), so key descending,
 // then slot ascending) and writes the request's next state: the reorder
 // gathers and the next step's candidate offsets.  All threads of the block
 // (blockDim.x >= K) call it.
@@ -847,7 +900,7 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
             }
             if (child < 0) set_error(a.err, FR_ERR_DEVICE);
             a.nxt.node[oj] = child;
-            a.nxt.score[oj] = key_to_float(key);
+            a.nxt.score[oj] = (a.rank == a.cand) ? key_to_float(key) : a.cand[(int64_t)b * a.cand_stride + slot];
             a.nxt.kv[oj] = a.cur.kv[ok];
             a.parent_out[oj] = k;
             a.token_out[oj] = tok;
@@ -894,7 +947,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
         n = 0;
     }
     const int Kp = min(K, n);
-    const float* cb = a.cand + (int64_t)b * a.cand_stride;
+    const float* cb = a.rank + (int64_t)b * a.cand_stride;
 
     if (Kp > 0) {
         uint32_t va = 0xFFFFFFFFu, vo = 0u;
@@ -1036,7 +1089,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
         for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = off_row[i];
         if (tid == 0) s_misc[0] = 0;  // the leader's winner count
     }
-    const float* cb = a.cand + (int64_t)b * a.cand_stride + lo;
+    const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;
     uint32_t va = 0xFFFFFFFFu, vo = 0u;
     for (int i = tid; i < cnt; i += SEL_THREADS) {
         const uint32_t k = float_to_key(cb[i]);
@@ -1288,6 +1341,10 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.row_cnt = buf.row_cnt;
     a.err = buf.err;
     a.lse_out = nullptr;
+    a.cand_key = sh.inv_temp > 0.f ? buf.cand_key : nullptr;
+    a.inv_temp = sh.inv_temp;
+    a.gseed = sh.gseed;
+    a.req_offset = sh.req_offset;
     if (sh.norm == FR_NORM_CANDIDATES) {
         const dim3 grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
         k_slice_candidates<<<grid, 256, 0, s>>>(a);
@@ -1341,6 +1398,7 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
     a.D = sh.D;
     a.t = t;
     a.cand = buf.cand;
+    a.rank = sh.inv_temp > 0.f ? buf.cand_key : buf.cand;
     a.cand_stride = buf.cand_stride;
     a.parent_out = buf.parent;
     a.token_out = buf.token;

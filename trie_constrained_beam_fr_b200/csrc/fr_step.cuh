@@ -12,7 +12,8 @@ struct StepBuffers {
     StateDev st[2];
     int32_t* parent;      // [B*K] latest step
     int32_t* token;       // [B*K]
-    float* cand;          // [B * cand_stride]
+    float* cand;          // [B * cand_stride] candidate scores
+    float* cand_key;      // [B * cand_stride] perturbed keys (sampling above temperature 0)
     int64_t cand_stride;  // K * max_fanout
     float2* partial;      // [grid * 2] (max, scaled sum) per CTA and row side
     int32_t* row_cnt;     // [B*K] arrival counters of shared rows
@@ -27,6 +28,9 @@ struct StepShape {
     int32_t sid_span;  // C_0 + ... + C_{D-1}: width of the SID token range
     int32_t sel_cluster[FR_MAX_DEPTH];  // per step: CTAs per request of the cluster select (0: one CTA)
     int64_t sel_bound[FR_MAX_DEPTH];    // per step: most candidates a request can have
+    float inv_temp;      // 1 / temperature; 0 = deterministic top-K
+    uint64_t gseed;      // Gumbel stream seed
+    int64_t req_offset;  // index of local request 0 in the Gumbel stream
 };
 
 // Cluster size of the selection for a step whose requests have at most

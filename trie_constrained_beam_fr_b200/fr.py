@@ -58,6 +58,7 @@ FR_FUNCS = [
     ("fr_beam_get_state", _I32, [_VP, _P(_I32), _VP, _VP, _VP, _VP, _VP]),
     ("fr_beam_set_state", _I32, [_VP, _I32, _VP, _VP, _VP, _VP, _VP]),
     ("fr_beam_set_normalization", _I32, [_VP, _I32]),
+    ("fr_beam_set_sampling", _I32, [_VP, ctypes.c_float, _U64, _I64]),
     ("fr_beam_set_timing", _I32, [_VP, _I32]),
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
@@ -267,6 +268,11 @@ def fr_beam_set_state(beam, steps_done: int, live: np.ndarray, prefix: np.ndarra
 
 def fr_beam_set_normalization(beam, norm: int) -> None:
     _check(libfr().fr_beam_set_normalization(beam, int(norm)), "fr_beam_set_normalization")
+
+
+def fr_beam_set_sampling(beam, temperature: float, seed: int = 0, request_offset: int = 0) -> None:
+    _check(libfr().fr_beam_set_sampling(beam, float(temperature), int(seed) & 0xFFFFFFFFFFFFFFFF,
+                                        int(request_offset)), "fr_beam_set_sampling")
 
 
 def fr_beam_set_timing(beam, enable: bool) -> None:
