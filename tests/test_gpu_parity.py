@@ -16,12 +16,19 @@ from frlib import GpuBeam, check_invariants, compare_step, near_tie_in, oracle_c
 pytestmark = pytest.mark.gpu
 
 W = synth.Workload
+# Rows whose streamed window is at most 16 KB take the warp-per-row kernel
+# (tiny, ragged_bf16, k1024, greedy, k_exceeds_catalog, k1024_wide_fanout);
+# longer rows take the persistent streaming kernel (ragged_wide_bf16,
+# mid_bf16, mid_f32_deep, full_vocab_few_rows, skewed_small).
 SMALL = {
     # the tiny workload itself
     "tiny": synth.WORKLOADS["tiny"],
     # bf16, V not a multiple of 8, SID range not 16-byte aligned, 3 requests
     "ragged_bf16": W("ragged_bf16", B=3, K=16, depth=3, C=16, V=1003, sid_base=13, n_items=2000, dtype="bf16",
                      seed=11, catalog_seed=11),
+    # the same raggedness on rows long enough for the streaming kernel
+    "ragged_wide_bf16": W("ragged_wide_bf16", B=3, K=16, depth=3, C=16, V=10003, sid_base=13, n_items=2000,
+                          dtype="bf16", seed=12, catalog_seed=12),
     # rows of 20000 spread over ~1.7 CTAs each: cross-CTA partials
     "mid_bf16": W("mid_bf16", B=4, K=64, depth=3, C=64, V=20000, sid_base=1000, n_items=20000, dtype="bf16",
                   seed=2, catalog_seed=2),
@@ -167,9 +174,10 @@ def test_single_child_chain_trie():
         np.testing.assert_array_equal(g_items[b], ref.items[b])
 
 
+@pytest.mark.parametrize("name", ["ragged_bf16", "ragged_wide_bf16"])
 @pytest.mark.parametrize("misalign,ld_pad", [(1, 0), (0, 5), (3, 7)])
-def test_strided_and_unaligned_rows(misalign, ld_pad):
-    w = SMALL["ragged_bf16"]
+def test_strided_and_unaligned_rows(misalign, ld_pad, name):
+    w = SMALL[name]
     sids = _catalog(w)
     ref = oracle.decode(oracle_cfg(w), oracle.Catalog(sids, w.codebook_sizes))
     gpu = GpuBeam(w, sids, ld=w.V + ld_pad, misalign=misalign)
@@ -223,8 +231,9 @@ def test_kv_slots_follow_parents():
         prev_kv = v.kv
 
 
+@pytest.mark.parametrize("V", [40000, 4000])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_extreme_logit_ranges(dtype):
+def test_extreme_logit_ranges(dtype, V):
     """Rows whose maximum comes late, jumps far above the first values, or
     follows a run of -inf: the streaming log-sum-exp moves its reference point
     (and re-sums a chunk when a term could overflow).  Expected scores are
@@ -232,8 +241,8 @@ def test_extreme_logit_ranges(dtype):
     import torch
     from scipy.special import logsumexp
 
-    V, C = 40000, 64
-    w = W("extreme", B=4, K=16, depth=1, C=C, V=V, sid_base=30000, n_items=C, dtype=dtype)
+    C = 64
+    w = W("extreme", B=4, K=16, depth=1, C=C, V=V, sid_base=V * 3 // 4, n_items=C, dtype=dtype)
     sids = np.arange(C, dtype=np.int32).reshape(-1, 1)
     gpu = GpuBeam(w, sids)
     try:
@@ -241,8 +250,8 @@ def test_extreme_logit_ranges(dtype):
         rows = np.stack([
             -150.0 + 300.0 * v / V,                                  # rising ramp, max at the end
             150.0 - 300.0 * v / V,                                   # falling ramp
-            np.where(v == 35000, 100.0, -50.0 + (v % 7) * 0.25),      # late spike far above the rest
-            np.where(v < 20000, -np.inf, np.sin(v) * 3.0),           # long run of -inf first
+            np.where(v == V * 7 // 8, 100.0, -50.0 + (v % 7) * 0.25),  # late spike far above the rest
+            np.where(v < V // 2, -np.inf, np.sin(v) * 3.0),            # long run of -inf first
         ])
         t = torch.tensor(rows, dtype=torch.float32)
         t = t.to(torch.bfloat16) if dtype == "bf16" else t

@@ -1,7 +1,9 @@
 // fr_step.cu -- the trie-constrained beam-search step on sm_100a.
 //
 // One step ("beamgrad 2.0.0 PKG-INFO", first code example and §Features;
-// "flashrec 0.1.1 METADATA", §Features/Decoding) is two kernels:
+// "flashrec 0.1.1 METADATA", §Features/Decoding) is two kernels (rows of at
+// most 16 KB take k_rows_short, a warp per row, in place of k_stream; the
+// candidate-slice normalisation takes k_slice_candidates):
 //
 //  k_stream  log-sum-exp of every live logits row over the full vocabulary,
 //            then, for each row, the trie children's candidate scores
@@ -80,6 +82,17 @@ constexpr int POLY_PAIRS = FR_POLY_PAIRS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
+
+// Programmatic dependent launch (sm_90 and later).  The step kernels are
+// launched with programmatic stream serialization, so a kernel may be
+// scheduled while the previous kernel of the stream is still running: it first
+// waits (griddep_wait) until that kernel has completed and its memory is
+// visible, then allows the next kernel to be scheduled
+// (griddep_launch_dependents).  The next kernel is released only once every
+// CTA of this one has signalled, so it never takes resources this grid still
+// needs.  For a kernel launched without the attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 struct Job {
     int64_t r;  // row whose segment in this CTA is reduced
@@ -551,6 +564,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
     SmemHdr* hdr = reinterpret_cast<SmemHdr*>(smem + RING_BYTES);
     int32_t* row_start = reinterpret_cast<int32_t*>(hdr + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (warp == 0) {  // row_start = exclusive scan of the live counts
         const int per = (a.B + 31) / 32;
@@ -739,6 +754,69 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
 }
 
 // ---------------------------------------------------------------------------
+// Short rows: when a row's streamed window is at most SHORT_ROW_BYTES (the SID
+// token range, or a small vocabulary) the persistent kernel's per-segment
+// bookkeeping costs more than the bytes.  One warp per live row instead: the
+// window's 16-byte-aligned interior in lane-interleaved batches of VPL
+// vectors per lane (2 KB per warp, all loads of a batch in flight together),
+// each batch's maximum first and then its exponent sum against the running
+// maximum (so no term can overflow); the unaligned head and tail as single
+// elements.  The row is then finished like any other (finish_row).
+
+constexpr int64_t SHORT_ROW_BYTES = 16384;
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
+    constexpr int ELT = BF16 ? 2 : 4;
+    constexpr int64_t VE = 16 / ELT;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    const int k = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int live = min(max(a.live[b], 0), a.K);
+    if (k >= live) return;
+    Seg sg;
+    sg.b = b;
+    sg.k = k;
+    sg.row = a.logits + ((int64_t)b * a.K + k) * a.ld * ELT;
+    sg.ptr = sg.row + a.col0 * ELT;
+    const int64_t W = a.W;
+    const uint32_t mis = (uint32_t)reinterpret_cast<uint64_t>(sg.ptr) & 15u;
+    const int64_t a0 = min((int64_t)((16u - mis) & 15u) / ELT, W);
+    const int64_t nvec = (W - a0) / VE;
+    const int64_t a1 = a0 + nvec * VE;
+    const uint4* vec = reinterpret_cast<const uint4*>(sg.ptr + a0 * ELT);
+    const uint32_t ninf = BF16 ? 0xFF80FF80u : 0xFF800000u;
+    const uint4 ninf4 = make_uint4(ninf, ninf, ninf, ninf);
+
+    float m = -INFINITY;
+    f32x2 s2 = 0ull;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * VPL) {
+        uint4 q[VPL];
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int64_t i = v0 + j * 32 + lane;
+            q[j] = i < nvec ? __ldg(vec + i) : ninf4;
+        }
+        const float mn = fmax_nan(m, lane_max<BF16>(q));
+        if (m != -INFINITY && mn != m) {
+            const float sc = ex2_approx((m - mn) * L2E);  // NaN when mn is NaN
+            s2 = mul2(s2, pack2(sc, sc));
+        }
+        m = mn;
+        if (m != -INFINITY) s2 = add2(s2, lane_expsum<BF16, 0>(q, m));
+    }
+    for (int64_t i = lane; i < a0; i += 32) lane_add(m, s2, load_elem(sg.ptr, i, ELT));
+    for (int64_t i = a1 + lane; i < W; i += 32) lane_add(m, s2, load_elem(sg.ptr, i, ELT));
+    float lo, hi;
+    unpack2(s2, lo, hi);
+    float s = lo + hi;
+    warp_combine(m, s);
+    finish_row<false>(a, sg, m, s);
+}
+
+// ---------------------------------------------------------------------------
 // Candidate-slice normalisation ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation
 // step 4: probabilities over the candidate slice): a beam's log-softmax runs
 // over its allowed children only, so no logits row is streamed.  One warp per
@@ -746,6 +824,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
 // the candidate scores s_k + (x - lse_slice).
 
 __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.x;
     const int k = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -793,6 +873,7 @@ constexpr int HBITS = 12;
 constexpr int HBINS = 1 << HBITS;
 static_assert(HBINS == 4 * SEL_THREADS, "each thread owns four histogram bins");
 static_assert(FR_MAX_K <= SEL_THREADS, "one thread per beam slot");
+static_assert(HBINS * sizeof(int32_t) >= FR_MAX_K * sizeof(unsigned long long), "histogram doubles as sort scratch");
 
 struct SelectArgs {
     StateDev cur, nxt;
@@ -847,30 +928,52 @@ __device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, 
 // then slot ascending) and writes the request's next state: the reorder
 // gathers and the next step's candidate offsets.  All threads of the block
 // (blockDim.x >= K) call it.
+// Sorts the n (<= blockDim.x) distinct nonzero values sel[0..n) into
+// descending order: a bitonic network over P = max(32, next power of two >= n)
+// values held one per thread by threads 0..P-1, padded with 0 (below every
+// real value).  Compare-exchange partners closer than 32 are in the same warp
+// (shuffles); the farther ones exchange through shared memory, alternating
+// between `buf` (P values of scratch) and sel so that each such stage needs
+// one barrier, a named barrier over the P participating threads only.  All
+// threads of the block call it.
+__device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ void sort_desc_u64(unsigned long long* sel, unsigned long long* buf, int n) {
+    const int tid = threadIdx.x;
+    int P = 32;
+    while (P < n) P <<= 1;
+    if (tid < P) {  // whole warps: P is a multiple of 32
+        unsigned long long v = tid < n ? sel[tid] : 0ull;
+        int par = 0;
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                unsigned long long o;
+                if (j >= 32) {
+                    unsigned long long* x = par ? sel : buf;
+                    x[tid] = v;
+                    bar_sync_named(1, P);
+                    o = x[tid ^ j];
+                    par ^= 1;
+                } else {
+                    o = __shfl_xor_sync(0xffffffffu, v, j);
+                }
+                const bool keep_max = ((tid & j) == 0) == ((tid & k) == 0);
+                v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+            }
+        }
+        bar_sync_named(1, P);
+        if (tid < n) sel[tid] = v;
+    }
+    __syncthreads();
+}
+
 __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, int Kp,
-                                 unsigned long long* sel) {
+                                 unsigned long long* sel, unsigned long long* scratch) {
     const int tid = threadIdx.x;
     const int K = a.K, D = a.D, t = a.t;
-    int P = 1;
-    while (P < Kp) P <<= 1;
-    for (int i = Kp + tid; i < P; i += blockDim.x) sel[i] = 0ull;
-    __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += blockDim.x) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const unsigned long long x = sel[i], y = sel[ixj];
-                    const bool swap = ((i & k) == 0) ? (x < y) : (x > y);
-                    if (swap) {
-                        sel[i] = y;
-                        sel[ixj] = x;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    sort_desc_u64(sel, scratch, Kp);
 
     // emit survivors (thread j = slot j)
     const int j = tid;
@@ -931,13 +1034,15 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
 
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
     __shared__ int32_t s_off[FR_MAX_K + 1];
-    __shared__ int32_t hist[HBINS];
+    __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
     __shared__ unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_misc[4];
     __shared__ uint32_t red[64];
     const int b = blockIdx.x, tid = threadIdx.x;
-    const int K = a.K, D = a.D, t = a.t;
+    const int K = a.K;
     const int live = min(max(a.cur.live[b], 0), K);
     for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
     __syncthreads();
@@ -949,10 +1054,27 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     const int Kp = min(K, n);
     const float* cb = a.rank + (int64_t)b * a.cand_stride;
 
-    if (Kp > 0) {
+    if (Kp > 0 && Kp == n) {
+        // every candidate survives: no threshold to find
+        for (int i = tid; i < n; i += SEL_THREADS)
+            sel[i] = ((unsigned long long)float_to_key(__ldg(cb + i)) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+        __syncthreads();
+    } else if (Kp > 0) {
         uint32_t va = 0xFFFFFFFFu, vo = 0u;
-        for (int i = tid; i < n; i += SEL_THREADS) {
-            const uint32_t k = float_to_key(cb[i]);
+        int i0 = tid;
+        for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
+            float x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t k = float_to_key(x[u]);
+                va &= k;
+                vo |= k;
+            }
+        }
+        for (int i = i0; i < n; i += SEL_THREADS) {
+            const uint32_t k = float_to_key(__ldg(cb + i));
             va &= k;
             vo |= k;
         }
@@ -977,8 +1099,19 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
                 for (int i = tid; i < HBINS; i += SEL_THREADS) hist[i] = 0;
                 __syncthreads();
                 const uint64_t want = (uint64_t)prefix >> lo;
-                for (int i = tid; i < n; i += SEL_THREADS) {
-                    const uint32_t k = float_to_key(cb[i]);
+                int i0 = tid;
+                for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
+                    float x[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t k = float_to_key(x[u]);
+                        if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
+                    }
+                }
+                for (int i = i0; i < n; i += SEL_THREADS) {
+                    const uint32_t k = float_to_key(__ldg(cb + i));
                     if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
                 }
                 __syncthreads();
@@ -1016,7 +1149,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
         __syncthreads();
         if (eq_needed >= count_eq) {
             for (int i = tid; i < n; i += SEL_THREADS) {
-                const uint32_t k = float_to_key(cb[i]);
+                const uint32_t k = float_to_key(__ldg(cb + i));
                 if (k >= T) {
                     const int p = atomicAdd(&s_misc[3], 1);
                     if (p < FR_MAX_K) sel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
@@ -1026,7 +1159,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
             int run_eq = 0;
             for (int base = 0; base < n; base += SEL_THREADS) {
                 const int i = base + tid;
-                const uint32_t k = i < n ? float_to_key(cb[i]) : 0u;
+                const uint32_t k = i < n ? float_to_key(__ldg(cb + i)) : 0u;
                 const bool gt = i < n && k > T;
                 const bool eq = i < n && k == T;
                 int tot;
@@ -1041,7 +1174,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
         __syncthreads();
         if (tid == 0 && s_misc[3] != Kp) set_error(a.err, FR_ERR_DEVICE);
     }
-    select_sort_emit(a, b, live, s_off, Kp, sel);
+    select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
 // ---------------------------------------------------------------------------
@@ -1061,6 +1194,8 @@ namespace cg = cooperative_groups;
 constexpr int CSEL_MAXKEYS = 40960;  // keys per CTA (160 KB of shared memory)
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
     cg::cluster_group cl = cg::this_cluster();
     extern __shared__ __align__(16) uint32_t keys[];
     __shared__ __align__(16) int32_t hist[2][HBINS];
@@ -1091,8 +1226,21 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     }
     const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;
     uint32_t va = 0xFFFFFFFFu, vo = 0u;
-    for (int i = tid; i < cnt; i += SEL_THREADS) {
-        const uint32_t k = float_to_key(cb[i]);
+    int i0 = tid;
+    for (; i0 + 7 * SEL_THREADS < cnt; i0 += 8 * SEL_THREADS) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t k = float_to_key(x[u]);
+            keys[i0 + u * SEL_THREADS] = k;
+            va &= k;
+            vo |= k;
+        }
+    }
+    for (int i = i0; i < cnt; i += SEL_THREADS) {
+        const uint32_t k = float_to_key(__ldg(cb + i));
         keys[i] = k;
         va &= k;
         vo |= k;
@@ -1115,7 +1263,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     int eq_needed = 0, count_eq = 0, eq_before = 0;
     if (Kp > 0) {
         const uint32_t diff = GA ^ GO;
-        if (diff == 0u) {
+        if (Kp == n) {
+            // every candidate survives: every key is >= 0 and all are taken
+            T = 0u;
+            eq_needed = count_eq = n;
+        } else if (diff == 0u) {
             T = GA;
             eq_needed = Kp;
             count_eq = n;
@@ -1214,7 +1366,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     cl.sync();
     if (c != 0) return;
     if (tid == 0 && s_misc[0] != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(a, b, live, s_off, Kp, sel);
+    select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
 // ---------------------------------------------------------------------------
@@ -1284,6 +1436,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_cand_off(StateDev st, int32_t K
 
 __global__ void k_finalize(StateDev st, int32_t B, int32_t K, int32_t D, TrieDev trie, int32_t* __restrict__ sids,
                            float* __restrict__ scores, int32_t* __restrict__ items) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t nbk = (int64_t)B * K;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
         const int32_t node = st.node[i];
@@ -1298,6 +1452,34 @@ __global__ void k_finalize(StateDev st, int32_t B, int32_t K, int32_t D, TrieDev
         }
     }
 }
+
+// Launch configuration of a step kernel: programmatic stream serialization
+// (see griddep_wait), and optionally a cluster size.  Used in place (cfg
+// points into the object).
+struct StepLaunch {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[2];
+    StepLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster = 0) {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        int n = 1;
+        if (cluster) {
+            attr[1].id = cudaLaunchAttributeClusterDimension;
+            attr[1].val.clusterDim.x = cluster;
+            attr[1].val.clusterDim.y = 1;
+            attr[1].val.clusterDim.z = 1;
+            n = 2;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = n;
+    }
+    StepLaunch(const StepLaunch&) = delete;
+    StepLaunch& operator=(const StepLaunch&) = delete;
+};
 
 int small_grid(int64_t n) {
     const int64_t g = (n + 255) / 256;
@@ -1345,17 +1527,19 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.inv_temp = sh.inv_temp;
     a.gseed = sh.gseed;
     a.req_offset = sh.req_offset;
+    const dim3 warp_grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
     if (sh.norm == FR_NORM_CANDIDATES) {
-        const dim3 grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
-        k_slice_candidates<<<grid, 256, 0, s>>>(a);
-        return cudaGetLastError();
+        StepLaunch L(warp_grid, 256, 0, s);
+        return cudaLaunchKernelEx(&L.cfg, k_slice_candidates, a);
     }
-    const size_t smem = stream_smem_bytes(sh.B);
-    if (sh.dtype == FR_BF16)
-        k_stream<true, false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
-    else
-        k_stream<false, false><<<sh.grid, STREAM_THREADS, smem, s>>>(a);
-    return cudaGetLastError();
+    if ((int64_t)a.W * a.elt <= SHORT_ROW_BYTES) {
+        StepLaunch L(warp_grid, 256, 0, s);
+        return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_rows_short<true>, a)
+                                   : cudaLaunchKernelEx(&L.cfg, k_rows_short<false>, a);
+    }
+    StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B), s);
+    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true, false>, a)
+                               : cudaLaunchKernelEx(&L.cfg, k_stream<false, false>, a);
 }
 
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
@@ -1405,23 +1589,12 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
     a.err = buf.err;
     const int cs = sh.sel_cluster[t];
     if (cs <= 0) {
-        k_select<<<sh.B, SEL_THREADS, 0, s>>>(a);
-        return cudaGetLastError();
+        StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, 0, s);
+        return cudaLaunchKernelEx(&L.cfg, k_select, a);
     }
     a.key_cap = (int32_t)((sh.sel_bound[t] + cs - 1) / cs);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sh.B * cs));
-    cfg.blockDim = dim3(SEL_THREADS);
-    cfg.dynamicSmemBytes = (size_t)a.key_cap * sizeof(uint32_t);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_select_cluster, a);
+    StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, (size_t)a.key_cap * sizeof(uint32_t), s, (unsigned)cs);
+    return cudaLaunchKernelEx(&L.cfg, k_select_cluster, a);
 }
 
 int select_cluster_size(int32_t B, int64_t bound, int32_t sms) {
@@ -1494,8 +1667,8 @@ cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const 
 cudaError_t launch_finalize(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, int32_t* sids,
                             float* scores, int32_t* items, cudaStream_t s) {
     const int64_t nbk = (int64_t)sh.B * sh.K;
-    k_finalize<<<small_grid(nbk), 256, 0, s>>>(buf.st[t & 1], sh.B, sh.K, sh.D, trie, sids, scores, items);
-    return cudaGetLastError();
+    StepLaunch L(dim3((unsigned)small_grid(nbk)), 256, 0, s);
+    return cudaLaunchKernelEx(&L.cfg, k_finalize, buf.st[t & 1], sh.B, sh.K, sh.D, trie, sids, scores, items);
 }
 
 }  // namespace fr
