@@ -15,7 +15,7 @@
 //            one producer lane moves 32 KB chunks from HBM into a 6-stage
 //            shared-memory ring with 1-D bulk async copies completing on
 //            mbarriers; 16 consumer warps each reduce a 2 KB slice of every
-//            chunk (running max + scaled exp2 sum per lane).  At the end of a
+//            chunk (running reference + scaled exp2 sum per lane).  At the end of a
 //            row segment the last consumer warp to arrive combines the 16
 //            warp partials in a fixed order and finishes the row; a row split
 //            across CTAs is finished by the last CTA to arrive (atomic
@@ -403,36 +403,35 @@ __device__ __forceinline__ float lane_max(const uint4 (&q)[VPL]) {
 // This lane's share (VPL 16-byte vectors, lane-interleaved) of one staged
 // chunk (already in registers; lanes past the chunk's end hold -inf), folded
 // into its running (reference m, packed scaled sum s2), where
-// sum exp(x) = exp(m) * (s2.lo + s2.hi).  The exponents are taken against
-// the reference the lane already holds (or its first element), so they do not
-// wait for the chunk's maximum; the maximum, computed alongside, moves the
-// reference afterwards when it rose by more than 16 (nats), and in the rare
-// case that it rose by more than 80 -- where a term could overflow -- the
-// chunk is summed again against the new maximum.
+// sum exp(x) = exp(m) * (s2.lo + s2.hi).  The exponents are taken against the
+// reference the lane already holds (its first element to begin with) and no
+// maximum is computed on the way: the reference only has to move when a term
+// could overflow, and the chunk's own sum shows that.  When the sum exceeds
+// 2^64, or is not finite (a term far above the reference, +inf or NaN in the
+// chunk, or an unusable -inf/NaN reference), the chunk's maximum becomes the
+// reference, the running sum is rescaled to it, and the chunk is summed again
+// (on the MUFU alone, which keeps NaN and infinities intact).  The reference
+// is always one of the values seen, so the sum is at least 1 and a term that
+// underflows to zero is below 2^-126 of it.
 template <bool BF16>
 __device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f32x2& s2) {
     float mref = m;
     if (mref == -INFINITY) mref = BF16 ? __uint_as_float(q[0].x << 16) : __uint_as_float(q[0].x);
     f32x2 part = lane_expsum<BF16, BF16 ? POLY_PAIRS : 0>(q, mref);
-    const float mx = lane_max<BF16>(q);
-    if (!(mref > -INFINITY && mx <= mref + 80.f)) {
-        // reference unusable (-inf/NaN first element), a term may overflow,
-        // or the chunk holds a NaN / +inf: sum again on the MUFU alone, which
-        // keeps NaN and infinities intact
-        mref = fmaxf(mx, mref);
+    float plo, phi;
+    unpack2(part, plo, phi);
+    if (!(mref > -INFINITY && plo + phi <= 0x1p64f)) {
+        const float mx = lane_max<BF16>(q);
+        const float mn = fmaxf(mx, mref);
         if (m != -INFINITY) {
-            const float sc = ex2_approx((m - mref) * L2E);
+            const float sc = ex2_approx((m - mn) * L2E);
             s2 = mul2(s2, pack2(sc, sc));
         }
-        part = lane_expsum<BF16, 0>(q, mref);
+        part = lane_expsum<BF16, 0>(q, mn);
+        mref = mn;
     }
     s2 = add2(s2, part);
     m = mref;
-    if (mx > m + 16.f) {
-        const float sc = ex2_approx((m - mx) * L2E);
-        s2 = mul2(s2, pack2(sc, sc));
-        m = mx;
-    }
 }
 
 // One element into a scalar (m, s): sum exp = exp(m) * s.
