@@ -107,6 +107,19 @@ fr_status fr_trie_level_sizes(const fr_trie* trie, int64_t* nodes_per_level);
 fr_status fr_trie_info(const fr_trie* trie, int32_t* depth, int32_t* sid_base,
                        int32_t* codebook_sizes, int32_t* max_fanout);
 
+/* Dense levels ("flashrec 0.1.1 METADATA", §Architecture: the fused kernel
+ * walks a dense or a CSR-sparse trie).  Level l is dense when every level-l
+ * node has all C_l children (nodes[l+1] == nodes[l] * C_l), detected at build
+ * time; the step kernels then index it directly (child of node n with code c
+ * = n * C_l + c) instead of reading child_off / code.  The CSR arrays are
+ * still built for every level.  dense_levels writes host int32 [depth]
+ * (1 = dense); set_dense(0) makes the kernels use the CSR arrays for every
+ * level, set_dense(1) (the default) uses direct indexing where a level is
+ * dense.  Results are identical either way.  Host-side; takes effect at the
+ * next kernel launch of any beam on this trie. */
+fr_status fr_trie_dense_levels(const fr_trie* trie, int32_t* dense_host);
+fr_status fr_trie_set_dense(fr_trie* trie, int32_t enable);
+
 /* Copies level l's CSR arrays to the host (synchronous; for tests and
  * inspection).  child_off_host: int32 [nodes[l] + 1] for l < depth, else must
  * be NULL; code_host: int32 [nodes[l]] for l >= 1, else must be NULL. */

@@ -48,6 +48,8 @@ def build_and_compare(sids: np.ndarray, C, sid_base=0):
             if l >= 1:
                 np.testing.assert_array_equal(cd, code[l])
         np.testing.assert_array_equal(fr.fr_trie_copy_leaf_rows(trie), rows)
+        # a level is dense when every one of its nodes has all C_l children
+        assert fr.fr_trie_dense_levels(trie) == [int(np.all(np.diff(child_off[l]) == C[l])) for l in range(len(C))]
     finally:
         fr.fr_trie_destroy(trie)
 

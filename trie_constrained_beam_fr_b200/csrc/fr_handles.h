@@ -14,6 +14,7 @@ struct fr_trie {
     int64_t nodes[FR_MAX_DEPTH + 1] = {};
     int32_t max_fanout = 0;
     int32_t level_fanout[FR_MAX_DEPTH] = {};  // largest child count of a level-l node
+    int32_t dense[FR_MAX_DEPTH] = {};         // level l is full: every node has all C_l children
     int32_t device = 0;
     int32_t* child_off[FR_MAX_DEPTH] = {};
     int32_t* code[FR_MAX_DEPTH + 1] = {};

@@ -22,8 +22,31 @@ struct TrieDev {
     const int32_t* leaf_row;                    // [nodes[depth]]
     int32_t nodes[FR_MAX_DEPTH + 1];
     int32_t tok_base[FR_MAX_DEPTH];             // token id of (level l, code 0)
+    // Dense levels ("flashrec 0.1.1 METADATA", §Architecture: dense or
+    // CSR-sparse trie): C_l when every level-l node has all C_l children (so
+    // child_off[l][n] = n * C_l and the child's code is its index mod C_l),
+    // else 0 (look the level up in the CSR arrays).
+    int32_t dense_c[FR_MAX_DEPTH];
     int32_t depth;
 };
+
+// Children of level-l node n: level-(l+1) node ids [lo, hi).
+__device__ __forceinline__ void trie_children(const TrieDev& t, int l, int32_t n, int32_t& lo, int32_t& hi) {
+    const int32_t c = t.dense_c[l];
+    if (c) {
+        lo = n * c;
+        hi = lo + c;
+    } else {
+        lo = t.child_off[l][n];
+        hi = t.child_off[l][n + 1];
+    }
+}
+
+// Code of level-(l+1) node m (a child of a level-l node).
+__device__ __forceinline__ int32_t trie_child_code(const TrieDev& t, int l, int32_t m) {
+    const int32_t c = t.dense_c[l];
+    return c ? m - (m / c) * c : t.code[l + 1][m];
+}
 
 // Beam state for one buffer of the double-buffered state.
 struct StateDev {

@@ -475,7 +475,8 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
         if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
         return;
     }
-    const int32_t lo = a.trie.child_off[t][n], hi = a.trie.child_off[t][n + 1];
+    int32_t lo, hi;
+    trie_children(a.trie, t, n, lo, hi);
     const int32_t base = a.cand_off[(int64_t)sg.b * (a.K + 1) + sg.k];
     if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) {
         if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
@@ -483,6 +484,7 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
     }
     const float sc = a.score[bk];
     const int32_t* codes = a.trie.code[t + 1] + lo;
+    const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
     const int32_t tb = a.trie.tok_base[t];
     float* out = a.cand + (int64_t)sg.b * a.cand_stride + base;
     const int32_t nch = hi - lo;
@@ -490,7 +492,7 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
         float* key = a.cand_key + (int64_t)sg.b * a.cand_stride + base;
         const uint64_t rh = gumbel_row_hash(a.gseed, a.req_offset + sg.b, t);
         for (int32_t i = lane; i < nch; i += 32) {
-            const int32_t tok = tb + __ldg(codes + i);
+            const int32_t tok = tb + (dense ? i : __ldg(codes + i));
             const float v = sc + (load_elem(sg.row, tok, a.elt) - lse);
             out[i] = v;
             key[i] = v * a.inv_temp + gumbel_noise(rh, sg.k, tok);
@@ -504,7 +506,7 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int32_t i = i0 + u * 32 + lane;
-            code[u] = i < nch ? __ldg(codes + i) : -1;
+            code[u] = i < nch ? (dense ? i : __ldg(codes + i)) : -1;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u], a.elt) : 0.f;
@@ -837,7 +839,8 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
         if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
         return;
     }
-    const int32_t lo = a.trie.child_off[t][n], hi = a.trie.child_off[t][n + 1];
+    int32_t lo, hi;
+    trie_children(a.trie, t, n, lo, hi);
     const int32_t base = a.cand_off[(int64_t)b * (a.K + 1) + k];
     if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) {
         if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
@@ -845,10 +848,12 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
     }
     const char* row = a.logits + bk * a.ld * a.elt;
     const int32_t* codes = a.trie.code[t + 1] + lo;
+    const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
     const int32_t tb = a.trie.tok_base[t];
     const int32_t nch = hi - lo;
     float m = -INFINITY, s = 0.f;
-    for (int32_t i = lane; i < nch; i += 32) lane_add_scalar(m, s, load_elem(row, tb + __ldg(codes + i), a.elt));
+    for (int32_t i = lane; i < nch; i += 32)
+        lane_add_scalar(m, s, load_elem(row, tb + (dense ? i : __ldg(codes + i)), a.elt));
     warp_combine(m, s);
     const float lse = m + logf(s);
     if (!isfinite(lse) && lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
@@ -857,7 +862,7 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
     float* key = a.cand_key ? a.cand_key + (int64_t)b * a.cand_stride + base : nullptr;
     const uint64_t rh = key ? gumbel_row_hash(a.gseed, a.req_offset + b, t) : 0ull;
     for (int32_t i = lane; i < nch; i += 32) {
-        const int32_t tok = tb + __ldg(codes + i);
+        const int32_t tok = tb + (dense ? i : __ldg(codes + i));
         const float v = sc + (load_elem(row, tok, a.elt) - lse);
         out[i] = v;
         if (key) key[i] = v * a.inv_temp + gumbel_noise(rh, k, tok);
@@ -915,7 +920,11 @@ __device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, 
     int cnt = 0;
     if (j < live) {
         const int32_t n = node_row[j];
-        if (n >= 0) cnt = trie.child_off[t_next][n + 1] - trie.child_off[t_next][n];
+        if (n >= 0) {
+            int32_t lo, hi;
+            trie_children(trie, t_next, n, lo, hi);
+            cnt = hi - lo;
+        }
     }
     int tot;
     const int e = block_excl_scan(cnt, &tot);
@@ -993,9 +1002,11 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
             const int32_t np = a.cur.node[ok];
             int32_t tok = -1;
             if (np >= 0 && np < a.trie.nodes[t]) {
-                child = a.trie.child_off[t][np] + (slot - s_off[k]);
+                int32_t lo, hi;
+                trie_children(a.trie, t, np, lo, hi);
+                child = lo + (slot - s_off[k]);
                 if (child >= 0 && child < a.trie.nodes[t + 1]) {
-                    tok = a.trie.tok_base[t] + a.trie.code[t + 1][child];
+                    tok = a.trie.tok_base[t] + trie_child_code(a.trie, t, child);
                 } else {
                     child = -1;
                 }
@@ -1022,7 +1033,11 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
         // node ids of the survivors are in registers of threads 0..Kp-1
         const int jj = threadIdx.x;
         int cnt = 0;
-        if (jj < Kp && child >= 0) cnt = a.trie.child_off[t + 1][child + 1] - a.trie.child_off[t + 1][child];
+        if (jj < Kp && child >= 0) {
+            int32_t lo, hi;
+            trie_children(a.trie, t + 1, child, lo, hi);
+            cnt = hi - lo;
+        }
         int tot;
         const int e = block_excl_scan(cnt, &tot);
         int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
@@ -1373,7 +1388,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
 
 __global__ void k_reset(StateDev s0, int32_t B, int32_t K, int32_t D, TrieDev trie) {
     const int64_t nbk = (int64_t)B * K;
-    const int32_t root_fan = trie.child_off[0][1] - trie.child_off[0][0];
+    int32_t root_lo, root_hi;
+    trie_children(trie, 0, 0, root_lo, root_hi);
+    const int32_t root_fan = root_hi - root_lo;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
         const int32_t b = (int32_t)(i / K), k = (int32_t)(i % K);
         const bool root = (k == 0);
@@ -1401,13 +1418,20 @@ __global__ void k_walk(StateDev st, int32_t B, int32_t K, int32_t D, int32_t t, 
             int32_t node = 0;
             for (int l = 0; l < t && node >= 0; ++l) {
                 const int32_t c = codes[i * D + l];
-                int32_t lo = trie.child_off[l][node], hi = trie.child_off[l][node + 1];
-                const int32_t* cl = trie.code[l + 1];
-                while (lo < hi) {  // first child with code >= c
-                    const int32_t mid = (lo + hi) >> 1;
-                    if (cl[mid] < c) lo = mid + 1; else hi = mid;
+                int32_t lo, end;
+                trie_children(trie, l, node, lo, end);
+                if (trie.dense_c[l]) {  // a full level: the child with code c is lo + c
+                    lo = (c >= 0 && c < trie.dense_c[l]) ? lo + c : end;
+                } else {
+                    const int32_t* cl = trie.code[l + 1];
+                    int32_t hi = end;
+                    while (lo < hi) {  // first child with code >= c
+                        const int32_t mid = (lo + hi) >> 1;
+                        if (cl[mid] < c) lo = mid + 1; else hi = mid;
+                    }
+                    if (lo < end && cl[lo] != c) lo = end;
                 }
-                if (lo < trie.child_off[l][node + 1] && cl[lo] == c) {
+                if (lo < end) {
                     node = lo;
                     st.prefix[i * D + l] = trie.tok_base[l] + c;
                 } else {

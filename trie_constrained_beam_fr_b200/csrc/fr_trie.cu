@@ -419,6 +419,12 @@ static fr_status trie_build_impl(const int32_t* sids, int64_t n, int32_t depth, 
         t->dev.nodes[l] = (int32_t)t->nodes[l];
     }
     t->dev.leaf_row = t->leaf_row;
+    // A level is full when it has nodes[l] * C_l children: every node then has
+    // all C_l codes, in code order.
+    for (int l = 0; l < depth; ++l) {
+        t->dense[l] = (t->nodes[l + 1] == t->nodes[l] * (int64_t)cb[l]) ? 1 : 0;
+        t->dev.dense_c[l] = t->dense[l] ? cb[l] : 0;
+    }
     return FR_OK;
 }
 
@@ -469,6 +475,18 @@ extern "C" fr_status fr_trie_info(const fr_trie* t, int32_t* depth, int32_t* sid
     if (cb)
         for (int l = 0; l < t->depth; ++l) cb[l] = t->codebook[l];
     if (max_fanout) *max_fanout = t->max_fanout;
+    return FR_OK;
+}
+
+extern "C" fr_status fr_trie_dense_levels(const fr_trie* t, int32_t* dense) {
+    if (!t || !dense) return FR_ERR_INVALID_ARG;
+    for (int l = 0; l < t->depth; ++l) dense[l] = t->dense[l];
+    return FR_OK;
+}
+
+extern "C" fr_status fr_trie_set_dense(fr_trie* t, int32_t enable) {
+    if (!t || (enable != 0 && enable != 1)) return FR_ERR_INVALID_ARG;
+    for (int l = 0; l < t->depth; ++l) t->dev.dense_c[l] = (enable && t->dense[l]) ? t->codebook[l] : 0;
     return FR_OK;
 }
 

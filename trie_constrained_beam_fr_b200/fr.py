@@ -45,6 +45,8 @@ FR_FUNCS = [
     ("fr_trie_build", _I32, [_VP, _I64, _I32, _P(_I32), _I32, _I32, _VP, _P(_VP)]),
     ("fr_trie_level_sizes", _I32, [_VP, _P(_I64)]),
     ("fr_trie_info", _I32, [_VP, _P(_I32), _P(_I32), _P(_I32), _P(_I32)]),
+    ("fr_trie_dense_levels", _I32, [_VP, _VP]),
+    ("fr_trie_set_dense", _I32, [_VP, _I32]),
     ("fr_trie_copy_level", _I32, [_VP, _I32, _VP, _VP]),
     ("fr_trie_copy_leaf_rows", _I32, [_VP, _VP]),
     ("fr_trie_destroy", None, [_VP]),
@@ -160,6 +162,17 @@ def fr_trie_info(trie) -> dict:
     cb = (_I32 * 16)()
     _check(libfr().fr_trie_info(trie, ctypes.byref(d), ctypes.byref(sb), cb, ctypes.byref(mf)), "fr_trie_info")
     return {"depth": d.value, "sid_base": sb.value, "codebook_sizes": list(cb)[: d.value], "max_fanout": mf.value}
+
+
+def fr_trie_dense_levels(trie) -> List[int]:
+    depth = fr_trie_info(trie)["depth"]
+    out = np.zeros(depth, dtype=np.int32)
+    _check(libfr().fr_trie_dense_levels(trie, out.ctypes.data), "fr_trie_dense_levels")
+    return out.tolist()
+
+
+def fr_trie_set_dense(trie, enable: bool) -> None:
+    _check(libfr().fr_trie_set_dense(trie, int(enable)), "fr_trie_set_dense")
 
 
 def fr_trie_copy_level(trie, level: int):
