@@ -29,6 +29,7 @@ NORM_CANDIDATES = 2
 MODE_HASH_F32 = 0
 MODE_HASH_BF16 = 1
 MODE_CONST = 2
+MODE_LMHEAD = 3
 
 ERR_NAMES = {0: "ok", 1: "invalid argument", 2: "duplicate SID", 3: "code out of range",
              4: "out of memory", 5: "not in catalog"}
@@ -55,7 +56,8 @@ class _Cfg(ctypes.Structure):
                 ("codebook", ctypes.c_int32 * 16), ("mode", ctypes.c_int32),
                 ("const_logit", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("b_offset", ctypes.c_int64), ("norm", ctypes.c_int32),
-                ("temperature", ctypes.c_double), ("gseed", ctypes.c_uint64)]
+                ("temperature", ctypes.c_double), ("gseed", ctypes.c_uint64),
+                ("hidden", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("hdim", ctypes.c_int32)]
 
 
 _lib = None
@@ -101,6 +103,10 @@ def lib():
         L.orc_decode.argtypes = [P(_Cfg), ctypes.c_void_p, P(ctypes.c_int32), P(ctypes.c_double),
                                  P(ctypes.c_int64), P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double),
                                  P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_double), P(ctypes.c_double)]
+        L.orc_lmhead_rows.restype = None
+        L.orc_lmhead_rows.argtypes = [P(ctypes.c_float), P(ctypes.c_float), ctypes.c_int64, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P(ctypes.c_double),
+                                      P(ctypes.c_double)]
         L.orc_gumbel.restype = ctypes.c_double
         L.orc_gumbel.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         L.orc_gen_seconds.restype = ctypes.c_double
@@ -153,6 +159,9 @@ class Config:
     norm: int = NORM_FULL
     temperature: float = 0.0
     gseed: int = 0
+    # MODE_LMHEAD: float32 arrays holding bf16 values, hidden [B, K, hdim], weight [V, hdim]
+    hidden: Optional[np.ndarray] = None
+    weight: Optional[np.ndarray] = None
 
     @classmethod
     def from_workload(cls, w, mode: Optional[int] = None, B: Optional[int] = None,
@@ -164,12 +173,38 @@ class Config:
 
     def c(self) -> _Cfg:
         cb = (ctypes.c_int32 * 16)(*([int(x) for x in self.codebook] + [0] * (16 - len(self.codebook))))
+        hid = wgt = None
+        hdim = 0
+        if self.mode == MODE_LMHEAD:
+            h = np.asarray(self.hidden)
+            wt = np.asarray(self.weight)
+            if (h.dtype != np.float32 or wt.dtype != np.float32 or not h.flags.c_contiguous
+                    or not wt.flags.c_contiguous or h.shape[:2] != (self.B, self.K) or wt.shape[0] != self.V
+                    or h.shape[2] != wt.shape[1]):
+                raise ValueError("lm_head mode needs float32 hidden [B, K, d] and weight [V, d]")
+            hid, wgt, hdim = h.ctypes.data, wt.ctypes.data, int(h.shape[2])
         return _Cfg(self.B, self.K, self.V, self.depth, self.sid_base, cb, self.mode,
                     self.const_logit, self.seed & 0xFFFFFFFFFFFFFFFF, self.b_offset, self.norm,
-                    float(self.temperature), self.gseed & 0xFFFFFFFFFFFFFFFF)
+                    float(self.temperature), self.gseed & 0xFFFFFFFFFFFFFFFF, hid, wgt, hdim)
 
     def token_base(self, level: int) -> int:
         return self.sid_base + int(sum(self.codebook[:level]))
+
+
+def lmhead_rows(h: np.ndarray, W: np.ndarray, sid_base: int, span: int):
+    """Per row of h [M, d]: log-sum-exp over all V of h . W^T (W [V, d]) and
+    the logits of columns [sid_base, sid_base + span), in double."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    M, d = h.shape
+    V = W.shape[0]
+    if W.shape[1] != d or sid_base < 0 or span < 0 or sid_base + span > V:
+        raise ValueError("bad lm_head shapes")
+    lse = np.empty(M, dtype=np.float64)
+    sl = np.empty((M, span), dtype=np.float64)
+    lib().orc_lmhead_rows(_ptr(h, ctypes.c_float), _ptr(W, ctypes.c_float), M, d, V, sid_base, span,
+                          _ptr(lse, ctypes.c_double), _ptr(sl, ctypes.c_double))
+    return lse, sl
 
 
 def fill_row(cfg: Config, b: int, tokens: Sequence[int]) -> np.ndarray:

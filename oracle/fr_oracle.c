@@ -72,6 +72,10 @@
 #define ORC_MODE_HASH_F32 0
 #define ORC_MODE_HASH_BF16 1
 #define ORC_MODE_CONST 2
+/* The row of slot k of request b is hidden[b, k, :] . weight[v, :] for every
+ * token v (the lm_head projection, "flashrec 0.1.1 METADATA",
+ * §Features/Decoding), accumulated in double from the given (bf16) values. */
+#define ORC_MODE_LMHEAD 3
 
 /* ------------------------------------------------------------------------- */
 /* SplitMix64 (Steele, Lea & Flood, OOPSLA 2014; Vigna's reference code).     */
@@ -145,6 +149,9 @@ typedef struct {
     int32_t norm;       /* ORC_NORM_*: the set the log-softmax normalises over */
     double temperature; /* 0: deterministic top-K; > 0: Gumbel top-K */
     uint64_t gseed;     /* seed of the Gumbel noise */
+    const float* hidden; /* ORC_MODE_LMHEAD: [B, K, hdim], local request index */
+    const float* weight; /* ORC_MODE_LMHEAD: [V, hdim] */
+    int32_t hdim;
 } orc_cfg;
 
 static int32_t level_token_base(const orc_cfg* cfg, int32_t level) {
@@ -175,6 +182,36 @@ double orc_row_lse(const float* x, int64_t V) {
     double s = 0.0;
     for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);
     return m + log(s);
+}
+
+/* The same over a double row. */
+static double row_lse_d(const double* x, int64_t n) {
+    double m = -INFINITY;
+    for (int64_t v = 0; v < n; ++v)
+        if (x[v] > m) m = x[v];
+    double s = 0.0;
+    for (int64_t v = 0; v < n; ++v) s += exp(x[v] - m);
+    return m + log(s);
+}
+
+/* lm_head rows: for each of the M rows of h [M, d], the logits
+ * x[v] = sum_j h[r, j] * W[v, j] (v < V) in double, their log-sum-exp over
+ * all V, and the logits of the SID token columns [sid_base, sid_base + span). */
+void orc_lmhead_rows(const float* h, const float* W, int64_t M, int32_t d, int32_t V, int32_t sid_base,
+                     int32_t span, double* lse, double* slice) {
+    double* x = (double*)malloc(sizeof(double) * (size_t)V);
+    for (int64_t r = 0; r < M; ++r) {
+        const float* hr = h + r * d;
+        for (int32_t v = 0; v < V; ++v) {
+            const float* wv = W + (int64_t)v * d;
+            double acc = 0.0;
+            for (int32_t j = 0; j < d; ++j) acc += (double)hr[j] * (double)wv[j];
+            x[v] = acc;
+        }
+        lse[r] = row_lse_d(x, V);
+        for (int32_t i = 0; i < span; ++i) slice[r * span + i] = x[sid_base + i];
+    }
+    free(x);
 }
 
 /* log of sum exp(x[idx[i]]) over the n given columns, in double. */
@@ -366,6 +403,7 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     const int32_t K = cfg->K, D = cfg->depth;
     if (t < 0 || t >= D || live < 0 || live > K) return -1;
     float* row = (float*)malloc(sizeof(float) * (size_t)cfg->V);
+    double* rowd = (double*)malloc(sizeof(double) * (size_t)cfg->V);
     int32_t cap = cfg->codebook[t];
     int32_t* kids = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
     int32_t* slice = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
@@ -376,23 +414,44 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
     for (int32_t k = 0; k < live; ++k) {
         for (int32_t l = 0; l < t; ++l) tokens[l] = level_token_base(cfg, l) + prefix[k * D + l];
         double t0 = now_seconds();
-        orc_fill_row(cfg, b, tokens, t, row);
+        const int lmhead = cfg->mode == ORC_MODE_LMHEAD;
+        if (lmhead) {
+            /* the slot's hidden state times every lm_head row, in double */
+            const float* hk = cfg->hidden + (b * (int64_t)K + k) * cfg->hdim;
+            for (int32_t v = 0; v < cfg->V; ++v) {
+                const float* wv = cfg->weight + (int64_t)v * cfg->hdim;
+                double acc = 0.0;
+                for (int32_t j = 0; j < cfg->hdim; ++j) acc += (double)hk[j] * (double)wv[j];
+                rowd[v] = acc;
+            }
+        } else {
+            orc_fill_row(cfg, b, tokens, t, row);
+            for (int32_t v = 0; v < cfg->V; ++v) rowd[v] = (double)row[v];
+        }
         g_gen_seconds += now_seconds() - t0;
         int32_t nk = orc_children(cat, prefix + k * D, t, kids, cap);
         double lse;
         if (cfg->norm == ORC_NORM_SID_RANGE) {
             int32_t span = 0;
             for (int32_t l = 0; l < D; ++l) span += cfg->codebook[l];
-            lse = orc_row_lse(row + cfg->sid_base, span);
+            lse = lmhead ? row_lse_d(rowd + cfg->sid_base, span) : orc_row_lse(row + cfg->sid_base, span);
         } else if (cfg->norm == ORC_NORM_CANDIDATES) {
             for (int32_t i = 0; i < nk; ++i) slice[i] = tok_base + kids[i];
-            lse = orc_subset_lse(row, slice, nk);
+            if (lmhead) {
+                double m = -INFINITY, sum = 0.0;
+                for (int32_t i = 0; i < nk; ++i)
+                    if (rowd[slice[i]] > m) m = rowd[slice[i]];
+                for (int32_t i = 0; i < nk; ++i) sum += exp(rowd[slice[i]] - m);
+                lse = m + log(sum);
+            } else {
+                lse = orc_subset_lse(row, slice, nk);
+            }
         } else {
-            lse = orc_row_lse(row, cfg->V);
+            lse = lmhead ? row_lse_d(rowd, cfg->V) : orc_row_lse(row, cfg->V);
         }
         for (int32_t i = 0; i < nk; ++i) {
             int32_t tok = tok_base + kids[i];
-            cand[nc].score = score[k] + ((double)row[tok] - lse);
+            cand[nc].score = score[k] + (rowd[tok] - lse);
             cand[nc].key = (cfg->temperature > 0.0)
                                ? cand[nc].score / cfg->temperature + orc_gumbel(cfg->gseed, b + cfg->b_offset, t, k, tok)
                                : cand[nc].score;
@@ -423,6 +482,7 @@ int32_t orc_step(const orc_cfg* cfg, const orc_catalog* cat, int64_t b, int32_t 
         }
     }
     free(row);
+    free(rowd);
     free(kids);
     free(slice);
     free(cand);

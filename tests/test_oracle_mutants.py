@@ -17,8 +17,16 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "fr_oracle.c")
 
 MUTANTS = {
-    "score_sign": ("cand[nc].score = score[k] + ((double)row[tok] - lse);",
-                   "cand[nc].score = score[k] - ((double)row[tok] - lse);"),
+    "score_sign": ("cand[nc].score = score[k] + (rowd[tok] - lse);",
+                   "cand[nc].score = score[k] - (rowd[tok] - lse);"),
+    "lmhead_step_wrong_weight_column": ("for (int32_t j = 0; j < cfg->hdim; ++j) acc += (double)hk[j] * (double)wv[j];",
+                                        "for (int32_t j = 0; j < cfg->hdim; ++j) acc += (double)hk[j] * (double)wv[0];"),
+    "lmhead_step_wrong_slot": ("const float* hk = cfg->hidden + (b * (int64_t)K + k) * cfg->hdim;",
+                               "const float* hk = cfg->hidden + (b * (int64_t)K) * cfg->hdim;"),
+    "lmhead_rows_transposed": ("for (int32_t j = 0; j < d; ++j) acc += (double)hr[j] * (double)wv[j];",
+                               "for (int32_t j = 0; j < d; ++j) acc += (double)hr[j] * (double)W[(int64_t)j * d + v % d];"),
+    "lmhead_slice_offset": ("for (int32_t i = 0; i < span; ++i) slice[r * span + i] = x[sid_base + i];",
+                            "for (int32_t i = 0; i < span; ++i) slice[r * span + i] = x[sid_base + i + 1];"),
     "lse_drops_max": ("for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);\n    return m + log(s);",
                       "for (int64_t v = 0; v < V; ++v) s += exp((double)x[v] - m);\n    return log(s);"),
     "subset_lse_drops_max": ("for (int32_t i = 0; i < n; ++i) s += exp((double)x[idx[i]] - m);\n    return m + log(s);",

@@ -487,3 +487,65 @@ def test_gumbel_vanishing_temperature_is_the_deterministic_beam():
     np.testing.assert_allclose(cold.scores, det.scores, atol=0)
     cfg.temperature = 0.0
     assert np.array_equal(oracle.decode(cfg, cat).step_key, det.step_score)
+
+
+# --------------------------------------------------------------------------
+# lm_head rows ("flashrec 0.1.1 METADATA", §Features/Decoding: the step's
+# logits are the lm_head projection of the beams' hidden states)
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_lmhead_rows_match_library_matmul_and_logsumexp():
+    rng = np.random.default_rng(5)
+    for M, d, V, sb, span in [(5, 64, 300, 100, 48), (3, 200, 1000, 0, 1000), (1, 8, 17, 16, 1)]:
+        h = _bf16(rng.standard_normal((M, d)))
+        W = _bf16(rng.standard_normal((V, d)) / np.sqrt(d))
+        lse, sl = oracle.lmhead_rows(h, W, sb, span)
+        x = h.astype(np.float64) @ W.astype(np.float64).T
+        np.testing.assert_allclose(lse, logsumexp(x, axis=1), atol=1e-10, rtol=0)
+        np.testing.assert_allclose(sl, x[:, sb: sb + span], atol=1e-10, rtol=0)
+
+
+def test_lmhead_rows_closed_form():
+    """Equal lm_head rows: every logit of a row is h . w, so the log-sum-exp is
+    h . w + ln V and the slice is constant."""
+    rng = np.random.default_rng(6)
+    d, V = 32, 500
+    h = _bf16(rng.standard_normal((4, d)))
+    w = _bf16(rng.standard_normal(d))
+    W = np.tile(w, (V, 1))
+    lse, sl = oracle.lmhead_rows(h, W, 100, 10)
+    x = h.astype(np.float64) @ w.astype(np.float64)
+    np.testing.assert_allclose(lse, x + math.log(V), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(sl, np.repeat(x[:, None], 10, axis=1), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("norm", [oracle.NORM_FULL, oracle.NORM_SID_RANGE, oracle.NORM_CANDIDATES])
+def test_lmhead_step_reduces_to_the_hash_step(norm):
+    """With lm_head = the identity (hdim = V) and each slot's hidden state set
+    to the hash logits row its prefix sees, the lm_head-mode step is the
+    hash-mode step, bit for bit, at every step of a decode."""
+    w, sids, cfg = _tiny_cfg(8, 500, oracle.MODE_HASH_BF16, seed=3, catalog_seed=3)
+    cfg.norm = norm
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    D, K, V = cfg.depth, cfg.K, cfg.V
+    eye = np.eye(V, dtype=np.float32)
+    prefix = np.full((K, D), -1, np.int32)
+    score = np.full(K, -np.inf)
+    score[0] = 0.0
+    live = 1
+    for t in range(D):
+        hidden = np.zeros((1, K, V), np.float32)
+        for k in range(live):
+            hidden[0, k] = oracle.fill_row(cfg, 0, [cfg.token_base(l) + prefix[k, l] for l in range(t)])
+        lm = oracle.Config(**{**cfg.__dict__, "mode": oracle.MODE_LMHEAD, "hidden": hidden, "weight": eye})
+        a = oracle.step(cfg, cat, 0, t, live, prefix, score)
+        b = oracle.step(lm, cat, 0, t, live, prefix, score)
+        assert a.live == b.live
+        np.testing.assert_array_equal(a.score, b.score)
+        np.testing.assert_array_equal(a.parent, b.parent)
+        np.testing.assert_array_equal(a.token, b.token)
+        prefix, score, live = a.prefix, a.score, a.live
