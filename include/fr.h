@@ -177,6 +177,30 @@ int32_t fr_beam_steps_done(const fr_beam* beam);
 fr_status fr_beam_finalize(fr_beam* beam, int32_t* sids_dev, float* scores_dev, int32_t* items_dev,
                            fr_stream stream);
 
+/* ------------------------------------------------------------------------- */
+/* lm_head fused with the row log-sum-exp ("flashrec 0.1.1 METADATA",         */
+/* §Features/Decoding: lm_head evaluated over the live beams' hidden states). */
+/*                                                                            */
+/* For rows h [rows, d] (bf16, row stride ldh elements) and lm_head W [V, d]  */
+/* (bf16, row stride ldw), computes on the tensor cores (fp32 accumulate)     */
+/*   lse[r]      = log sum_v exp(h_r . W_v)           (fp32, [rows])          */
+/*   slice[r][i] = h_r . W_{sid_base + i}, i < sid_span   (fp32, [rows, span])*/
+/* without writing the [rows, V] logits.  W is owned by the caller and must   */
+/* stay valid and unchanged for the handle's lifetime; h, lse and slice are   */
+/* the caller's device buffers.  Base pointers of h and W must be 16-byte     */
+/* aligned and ldh * 2, ldw * 2 multiples of 16 (FR_ERR_INVALID_ARG else).    */
+/* init allocates the partials for up to max_rows rows; run is stream-ordered */
+/* and asynchronous; status synchronises and returns the sticky device status */
+/* (FR_ERR_NAN_LOGIT for a non-finite row, FR_ERR_DEVICE on an internal       */
+/* timeout). */
+typedef struct fr_lmhead fr_lmhead;
+fr_status fr_lmhead_init(const void* weight_dev, int64_t ldw, int32_t V, int32_t d, int32_t max_rows,
+                         int32_t sid_base, int32_t sid_span, fr_lmhead** out);
+fr_status fr_lmhead_run(fr_lmhead* lmhead, const void* hidden_dev, int64_t ldh, int32_t rows, float* lse_dev,
+                        float* slice_dev, fr_stream stream);
+fr_status fr_lmhead_status(fr_lmhead* lmhead);
+void fr_lmhead_destroy(fr_lmhead* lmhead);
+
 /* Synchronises the beam's last stream and returns its sticky device status
  * (FR_OK, FR_ERR_NAN_LOGIT, FR_ERR_DEVICE, FR_ERR_NOT_IN_CATALOG) or FR_ERR_CUDA. */
 fr_status fr_beam_status(fr_beam* beam);

@@ -65,6 +65,10 @@ FR_FUNCS = [
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
     ("fr_row_logsumexp_noalloc", _I32, [_VP, _I64, _I32, _I32, _I32, _VP, _VP]),
+    ("fr_lmhead_init", _I32, [_VP, _I64, _I32, _I32, _I32, _I32, _I32, _P(_VP)]),
+    ("fr_lmhead_run", _I32, [_VP, _VP, _I64, _I32, _VP, _VP, _VP]),
+    ("fr_lmhead_status", _I32, [_VP]),
+    ("fr_lmhead_destroy", None, [_VP]),
 ]
 FR_GEN_FUNCS = [
     ("fr_gen_hash_logits", _I32, [_U64, _I64, _I32, _I32, _I32, _I64, _I32, _VP, _I32, _I32, _VP, _VP, _VP]),
@@ -335,3 +339,34 @@ def fr_gen_hash_logits(seed: int, b_offset: int, B: int, K: int, V: int, out: to
 def fr_gen_flush(buf: torch.Tensor, stream=None) -> None:
     _check(libfr_gen().fr_gen_flush(_dev_ptr(buf), buf.numel() * buf.element_size(), _stream(stream)),
            "fr_gen_flush")
+
+
+def fr_lmhead_init(weight: torch.Tensor, max_rows: int, sid_base: int, sid_span: int) -> ctypes.c_void_p:
+    """weight: bf16 [V, d] CUDA tensor (row stride weight.stride(0))."""
+    if weight.dtype != torch.bfloat16 or weight.dim() != 2 or weight.stride(1) != 1:
+        raise ValueError("weight must be a bf16 [V, d] CUDA tensor with unit column stride")
+    out = _VP()
+    st = libfr().fr_lmhead_init(_dev_ptr(weight), int(weight.stride(0)), int(weight.shape[0]), int(weight.shape[1]),
+                                int(max_rows), int(sid_base), int(sid_span), ctypes.byref(out))
+    _check(st, "fr_lmhead_init")
+    return out
+
+
+def fr_lmhead_run(lmhead, hidden: torch.Tensor, lse: torch.Tensor, slice_: Optional[torch.Tensor],
+                  stream=None) -> None:
+    """hidden: bf16 [rows, d]; lse: float32 [rows]; slice_: float32 [rows, sid_span]."""
+    if hidden.dtype != torch.bfloat16 or hidden.dim() != 2 or hidden.stride(1) != 1:
+        raise ValueError("hidden must be a bf16 [rows, d] CUDA tensor with unit column stride")
+    if lse.dtype != torch.float32 or (slice_ is not None and slice_.dtype != torch.float32):
+        raise ValueError("lse and slice must be float32")
+    st = libfr().fr_lmhead_run(lmhead, _dev_ptr(hidden), int(hidden.stride(0)), int(hidden.shape[0]),
+                               _dev_ptr(lse), None if slice_ is None else _dev_ptr(slice_), _stream(stream))
+    _check(st, "fr_lmhead_run")
+
+
+def fr_lmhead_status(lmhead) -> int:
+    return int(libfr().fr_lmhead_status(lmhead))
+
+
+def fr_lmhead_destroy(lmhead) -> None:
+    libfr().fr_lmhead_destroy(lmhead)
