@@ -201,6 +201,22 @@ fr_status fr_lmhead_run(fr_lmhead* lmhead, const void* hidden_dev, int64_t ldh, 
 fr_status fr_lmhead_status(fr_lmhead* lmhead);
 void fr_lmhead_destroy(fr_lmhead* lmhead);
 
+/* One beam step from given rows instead of logits (the lm_head path, §8 f1:
+ * the rows come from fr_lmhead_run).  Slot (b, k) reads row
+ * r = b * row_stride_b + k of
+ *   lse_dev    float [rows]            log-sum-exp of the row over the vocabulary
+ *   slice_dev  float [rows, sid_span]  logits of the SID tokens, column
+ *                                      v - sid_base for token v, where sid_span
+ *                                      = C_0 + ... + C_{depth-1}
+ * (device, caller-owned, read during the call's stream work).  Live slots
+ * must satisfy k < row_stride_b (e.g. row_stride_b = 1 at step 0, where only
+ * slot 0 is live, and K afterwards), else the device status becomes
+ * FR_ERR_DEVICE.  The normalisation set applies as in fr_beam_step: the full
+ * vocabulary uses lse_dev; the SID range and the candidate slice are
+ * normalised from slice_dev alone.  Otherwise as fr_beam_step. */
+fr_status fr_beam_step_lse(fr_beam* beam, const float* lse_dev, const float* slice_dev, int64_t row_stride_b,
+                           fr_stream stream);
+
 /* Synchronises the beam's last stream and returns its sticky device status
  * (FR_OK, FR_ERR_NAN_LOGIT, FR_ERR_DEVICE, FR_ERR_NOT_IN_CATALOG) or FR_ERR_CUDA. */
 fr_status fr_beam_status(fr_beam* beam);

@@ -187,6 +187,31 @@ extern "C" fr_status fr_beam_step(fr_beam* bm, const void* logits, int64_t ld, f
     return FR_OK;
 }
 
+extern "C" fr_status fr_beam_step_lse(fr_beam* bm, const float* lse, const float* slice, int64_t row_stride_b,
+                                      fr_stream stream) {
+    if (!bm || !lse || !slice || row_stride_b < 1) return FR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(slice) & 3u)) return FR_ERR_INVALID_ARG;
+    if (bm->t >= bm->shape.D) return FR_ERR_STATE;
+    const cudaStream_t s = (cudaStream_t)stream;
+    const bool timed = bm->timing && bm->n_timed < MAX_TIMED_STEPS;
+    cudaEvent_t* ev = timed ? &bm->events[3 * (size_t)bm->n_timed] : nullptr;
+    if (timed) {
+        for (int i = 0; i < 3; ++i)
+            if (!ev[i]) FR_CUDA_TRY(cudaEventCreate(&ev[i]));
+        FR_CUDA_TRY(cudaEventRecord(ev[0], s));
+    }
+    FR_CUDA_TRY(fr::launch_step_lse(bm->shape, bm->buf, bm->trie->dev, bm->t, lse, slice, row_stride_b, s));
+    if (timed) FR_CUDA_TRY(cudaEventRecord(ev[1], s));
+    FR_CUDA_TRY(fr::launch_select(bm->shape, bm->buf, bm->trie->dev, bm->t, s));
+    if (timed) {
+        FR_CUDA_TRY(cudaEventRecord(ev[2], s));
+        ++bm->n_timed;
+    }
+    ++bm->t;
+    bm->last_stream = s;
+    return FR_OK;
+}
+
 extern "C" fr_status fr_beam_outputs(const fr_beam* bm, const int32_t** parent, const int32_t** token,
                                      const int32_t** node, const float** score, const int32_t** kv_slot,
                                      const int32_t** live, const int32_t** prefix) {

@@ -128,6 +128,9 @@ struct StreamArgs {
     int32_t* row_cnt;
     int32_t* err;
     float* lse_out;  // log-sum-exp-only instantiation: lse of row (0, k) at lse_out[k]
+    int64_t row_stride_b;  // warp-per-row kernels: the row of slot (b, k) is b * row_stride_b + k
+    int32_t col_sub;       // the column of token v in a row is v - col_sub
+    const float* lse_in;   // step from given log-sum-exps: lse of slot (b, k) at its row index
     float* cand_key;     // sampling: perturbed keys beside cand (null at temperature 0)
     float inv_temp;      // 1 / temperature
     uint64_t gseed;      // seed of the Gumbel stream
@@ -456,15 +459,9 @@ __device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
 }
 
 // The row's log-sum-exp is known: write the scores of the trie children of
-// the row's beam.  One warp.
-template <bool LSE_ONLY>
-__device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
+// the row's beam (token v of the row at column v - col_sub).  One warp.
+__device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse) {
     const int lane = threadIdx.x & 31;
-    const float lse = m + logf(s);
-    if constexpr (LSE_ONLY) {
-        if (lane == 0) a.lse_out[sg.k] = lse;
-        return;
-    }
     if (!isfinite(lse)) {
         if (lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
     }
@@ -493,7 +490,7 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
         const uint64_t rh = gumbel_row_hash(a.gseed, a.req_offset + sg.b, t);
         for (int32_t i = lane; i < nch; i += 32) {
             const int32_t tok = tb + (dense ? i : __ldg(codes + i));
-            const float v = sc + (load_elem(sg.row, tok, a.elt) - lse);
+            const float v = sc + (load_elem(sg.row, tok - a.col_sub, a.elt) - lse);
             out[i] = v;
             key[i] = v * a.inv_temp + gumbel_noise(rh, sg.k, tok);
         }
@@ -509,13 +506,25 @@ __device__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s)
             code[u] = i < nch ? (dense ? i : __ldg(codes + i)) : -1;
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u], a.elt) : 0.f;
+        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u] - a.col_sub, a.elt) : 0.f;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int32_t i = i0 + u * 32 + lane;
             if (i < nch) out[i] = sc + (x[u] - lse);
         }
     }
+}
+
+// The row's (max, scaled sum) are known: its log-sum-exp, then its
+// candidates (or, LSE_ONLY, just the log-sum-exp).
+template <bool LSE_ONLY>
+__device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
+    const float lse = m + logf(s);
+    if constexpr (LSE_ONLY) {
+        if ((threadIdx.x & 31) == 0) a.lse_out[sg.k] = lse;
+        return;
+    }
+    finish_cands(a, sg, lse);
 }
 
 // Called by the warp that combined this CTA's partial for row r.
@@ -777,10 +786,14 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
     const int k = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int live = min(max(a.live[b], 0), a.K);
     if (k >= live) return;
+    if (k >= a.row_stride_b) {  // the caller's rows hold fewer slots than are live
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
     Seg sg;
     sg.b = b;
     sg.k = k;
-    sg.row = a.logits + ((int64_t)b * a.K + k) * a.ld * ELT;
+    sg.row = a.logits + ((int64_t)b * a.row_stride_b + k) * a.ld * ELT;
     sg.ptr = sg.row + a.col0 * ELT;
     const int64_t W = a.W;
     const uint32_t mis = (uint32_t)reinterpret_cast<uint64_t>(sg.ptr) & 15u;
@@ -818,6 +831,31 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Step from given log-sum-exps (the lm_head path: the row's log-sum-exp over
+// the vocabulary comes from the fused lm_head kernel and the row itself is
+// only its SID-range slice).  One warp per live slot.
+
+__global__ void __launch_bounds__(256) k_rows_given_lse(const StreamArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    const int k = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int live = min(max(a.live[b], 0), a.K);
+    if (k >= live) return;
+    if (k >= a.row_stride_b) {  // the caller's rows hold fewer slots than are live
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const int64_t r = (int64_t)b * a.row_stride_b + k;
+    Seg sg;
+    sg.b = b;
+    sg.k = k;
+    sg.row = a.logits + r * a.ld * a.elt;
+    finish_cands(a, sg, __ldg(a.lse_in + r));
+}
+
+// ---------------------------------------------------------------------------
 // Candidate-slice normalisation ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation
 // step 4: probabilities over the candidate slice): a beam's log-softmax runs
 // over its allowed children only, so no logits row is streamed.  One warp per
@@ -846,14 +884,19 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
         if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
         return;
     }
-    const char* row = a.logits + bk * a.ld * a.elt;
+    if (k >= a.row_stride_b) {  // the caller's rows hold fewer slots than are live
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
+    const char* row = a.logits + ((int64_t)b * a.row_stride_b + k) * a.ld * a.elt;
     const int32_t* codes = a.trie.code[t + 1] + lo;
     const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
-    const int32_t tb = a.trie.tok_base[t];
+    const int32_t tb = a.trie.tok_base[t];  // vocabulary id of the level's code 0
+    const int32_t cb = tb - a.col_sub;      // its column in the row
     const int32_t nch = hi - lo;
     float m = -INFINITY, s = 0.f;
     for (int32_t i = lane; i < nch; i += 32)
-        lane_add_scalar(m, s, load_elem(row, tb + (dense ? i : __ldg(codes + i)), a.elt));
+        lane_add_scalar(m, s, load_elem(row, cb + (dense ? i : __ldg(codes + i)), a.elt));
     warp_combine(m, s);
     const float lse = m + logf(s);
     if (!isfinite(lse) && lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
@@ -862,8 +905,9 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
     float* key = a.cand_key ? a.cand_key + (int64_t)b * a.cand_stride + base : nullptr;
     const uint64_t rh = key ? gumbel_row_hash(a.gseed, a.req_offset + b, t) : 0ull;
     for (int32_t i = lane; i < nch; i += 32) {
-        const int32_t tok = tb + (dense ? i : __ldg(codes + i));
-        const float v = sc + (load_elem(row, tok, a.elt) - lse);
+        const int32_t code = dense ? i : __ldg(codes + i);
+        const int32_t tok = tb + code;
+        const float v = sc + (load_elem(row, cb + code, a.elt) - lse);
         out[i] = v;
         if (key) key[i] = v * a.inv_temp + gumbel_noise(rh, k, tok);
     }
@@ -1550,6 +1594,9 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.inv_temp = sh.inv_temp;
     a.gseed = sh.gseed;
     a.req_offset = sh.req_offset;
+    a.row_stride_b = sh.K;
+    a.col_sub = 0;
+    a.lse_in = nullptr;
     const dim3 warp_grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
     if (sh.norm == FR_NORM_CANDIDATES) {
         StepLaunch L(warp_grid, 256, 0, s);
@@ -1563,6 +1610,44 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B), s);
     return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true, false>, a)
                                : cudaLaunchKernelEx(&L.cfg, k_stream<false, false>, a);
+}
+
+cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
+                            const float* lse, const float* slice, int64_t row_stride_b, cudaStream_t s) {
+    const StateDev& cur = buf.st[t & 1];
+    StreamArgs a{};
+    a.logits = reinterpret_cast<const char*>(slice);
+    a.ld = sh.sid_span;  // a row is the SID-range slice
+    a.V = sh.sid_span;
+    a.B = sh.B;
+    a.K = sh.K;
+    a.t = t;
+    a.elt = 4;
+    a.col0 = 0;
+    a.W = sh.sid_span;
+    a.live = cur.live;
+    a.node = cur.node;
+    a.score = cur.score;
+    a.cand_off = cur.cand_off;
+    a.trie = trie;
+    a.cand = buf.cand;
+    a.cand_stride = buf.cand_stride;
+    a.partial = buf.partial;
+    a.row_cnt = buf.row_cnt;
+    a.err = buf.err;
+    a.lse_out = nullptr;
+    a.row_stride_b = row_stride_b;
+    a.col_sub = trie.tok_base[0];  // token v of the SID range is column v - sid_base
+    a.lse_in = lse;
+    a.cand_key = sh.inv_temp > 0.f ? buf.cand_key : nullptr;
+    a.inv_temp = sh.inv_temp;
+    a.gseed = sh.gseed;
+    a.req_offset = sh.req_offset;
+    const dim3 warp_grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
+    StepLaunch L(warp_grid, 256, 0, s);
+    if (sh.norm == FR_NORM_CANDIDATES) return cudaLaunchKernelEx(&L.cfg, k_slice_candidates, a);
+    if (sh.norm == FR_NORM_SID_RANGE) return cudaLaunchKernelEx(&L.cfg, k_rows_short<false>, a);
+    return cudaLaunchKernelEx(&L.cfg, k_rows_given_lse, a);
 }
 
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,

@@ -49,6 +49,11 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
                            const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
                            cudaStream_t s);
+// The row phase of a step from given rows: slot (b, k) has the log-sum-exp
+// lse[b * row_stride_b + k] over the vocabulary and the SID-range logits
+// slice[(b * row_stride_b + k) * sid_span + (v - sid_base)].
+cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
+                            const float* lse, const float* slice, int64_t row_stride_b, cudaStream_t s);
 cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, cudaStream_t s);
 cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s);
 cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,

@@ -53,6 +53,7 @@ FR_FUNCS = [
     ("fr_beam_init", _I32, [_VP, _I32, _I32, _I32, _I32, _VP, _P(_VP)]),
     ("fr_beam_reset", _I32, [_VP, _VP]),
     ("fr_beam_step", _I32, [_VP, _VP, _I64, _VP]),
+    ("fr_beam_step_lse", _I32, [_VP, _VP, _VP, _I64, _VP]),
     ("fr_beam_outputs", _I32, [_VP] + [_P(_VP)] * 7),
     ("fr_beam_steps_done", _I32, [_VP]),
     ("fr_beam_finalize", _I32, [_VP, _VP, _VP, _VP, _VP]),
@@ -229,6 +230,14 @@ class _DeviceView:
     def __init__(self, ptr: int, shape, typestr: str):
         self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
                                          "version": 3, "strides": None, "stream": None}
+
+
+def fr_beam_step_lse(beam, lse: torch.Tensor, slice_: torch.Tensor, row_stride_b: int, stream=None) -> None:
+    """lse: float32 [rows]; slice_: float32 [rows, sid_span] (contiguous rows)."""
+    if lse.dtype != torch.float32 or slice_.dtype != torch.float32 or slice_.dim() != 2 or not slice_.is_contiguous():
+        raise ValueError("lse must be float32 [rows] and slice a contiguous float32 [rows, sid_span]")
+    _check(libfr().fr_beam_step_lse(beam, _dev_ptr(lse), _dev_ptr(slice_), int(row_stride_b), _stream(stream)),
+           "fr_beam_step_lse")
 
 
 def fr_beam_outputs(beam, B: int, K: int, depth: int) -> Dict[str, torch.Tensor]:

@@ -211,3 +211,39 @@ def workload_catalog(w: Workload) -> np.ndarray:
 def scaled(w: Workload, **kw) -> Workload:
     """A copy of ``w`` with some fields replaced (small parity variants)."""
     return dataclasses.replace(w, **kw)
+
+
+# ---------------------------------------------------------------------------
+# Synthetic lm_head inputs: hidden states of the beams and the lm_head matrix,
+# exact in bf16 (8 significant bits), for the lm_head path of the step.
+
+_HIDDEN_SALT = np.uint64(0x5EEDF00D5EEDF00D)
+_WEIGHT_SALT = np.uint64(0x0DDBA11CAFEF00D5)
+
+
+def _byte_values(u: np.ndarray, scale: float) -> np.ndarray:
+    """The top byte of each draw as a signed integer in [-128, 128), times a
+    power-of-two scale: exact in bf16 and in float32."""
+    return ((u >> np.uint64(56)).astype(np.int64) - 128).astype(np.float32) * np.float32(scale)
+
+
+def hidden_states(seed: int, b: int, prefixes, d: int) -> np.ndarray:
+    """float32 [len(prefixes), d]: the hidden state of request ``b`` after each
+    SID prefix (a sequence of token ids), values k / 64 with k in [-128, 128)."""
+    out = np.empty((len(prefixes), d), dtype=np.float32)
+    j = np.arange(d, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        for i, p in enumerate(prefixes):
+            h = splitmix64(np.uint64(seed) ^ _HIDDEN_SALT) ^ np.uint64(b)
+            for tok in p:
+                h = splitmix64(h ^ np.uint64(int(tok)))
+            out[i] = _byte_values(splitmix64(splitmix64(h) ^ j), 1.0 / 64)
+    return out
+
+
+def lm_head_weight(seed: int, V: int, d: int) -> np.ndarray:
+    """float32 [V, d], values k / 8192 with k in [-128, 128)."""
+    idx = np.arange(V * d, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        u = splitmix64(splitmix64(np.uint64(seed) ^ _WEIGHT_SALT) ^ idx)
+    return _byte_values(u, 1.0 / 8192).reshape(V, d)
