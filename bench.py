@@ -51,6 +51,9 @@ def parse_args():
                    help="log-softmax normalisation set (full vocabulary by default)")
     p.add_argument("--temperature", type=float, default=0.0,
                    help="0: deterministic top-K; > 0: Gumbel top-K sampling at this temperature")
+    p.add_argument("--lmhead", type=int, default=0, metavar="D",
+                   help="the lm_head path: hidden states of size D instead of logits (fused tensor-core "
+                        "lm_head + log-sum-exp, then the step from the SID-range slice)")
     return p.parse_args()
 
 
@@ -244,10 +247,179 @@ def run_reference(args):
 # GPU arm
 
 
+def run_lmhead(args):
+    """The lm_head path: per step, the live beams' hidden states [rows, D]
+    (bf16, random, resident in HBM) go through fr_lmhead_run (every row's
+    log-sum-exp over V and its SID-range logits, on the tensor cores) and
+    fr_beam_step_lse; one benchmark step is one full decode."""
+    import torch
+    import torch.distributed as dist
+
+    from trie_constrained_beam_fr_b200 import fr
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = synth.WORKLOADS[args.config]
+    if args.batch:
+        w = synth.scaled(w, B=args.batch)
+    B, K, D, V, dh = w.B, w.K, w.depth, w.V, args.lmhead
+    b_offset, _ = rank_requests(rank, world, B)
+    span = sum(w.codebook_sizes)
+    sids = torch.from_numpy(synth.workload_catalog(w)).to(dev)
+    trie = fr.fr_trie_build(sids, w.codebook_sizes, w.sid_base)
+    beam = fr.fr_beam_init(trie, B, K, V, "bf16")
+    fr.fr_beam_set_normalization(beam, NORM_CODES[args.norm])
+    if args.temperature > 0:
+        fr.fr_beam_set_sampling(beam, args.temperature, 0x5EED, b_offset)
+    g = torch.Generator(device=dev).manual_seed(1234 + rank)
+    weight = (torch.randn(V, dh, device=dev, generator=g) / dh ** 0.5).to(torch.bfloat16)
+    hidden = [torch.randn(B, K, dh, device=dev, generator=g).to(torch.bfloat16) for _ in range(D)]
+    lm = fr.fr_lmhead_init(weight, max_rows=B * K, sid_base=w.sid_base, sid_span=span)
+    lse = torch.empty(B * K, device=dev)
+    sl = torch.empty(B * K, span, device=dev)
+    out_sids = torch.empty((B, K, D), dtype=torch.int32, device=dev)
+    out_scores = torch.empty((B, K), dtype=torch.float32, device=dev)
+    out_items = torch.empty((B, K), dtype=torch.int32, device=dev)
+    rows_per_step = [B] + [B * K] * (D - 1)  # step 0: slot 0 of each request is the only live beam
+
+    def decode(hid, lm_events=None):
+        fr.fr_beam_reset(beam)
+        for t in range(D):
+            rows = rows_per_step[t]
+            h = hid[t][:, 0, :] if t == 0 else hid[t].view(B * K, dh)
+            if lm_events is not None:
+                lm_events[t][0].record()
+            fr.fr_lmhead_run(lm, h, lse[:rows], sl[:rows])
+            if lm_events is not None:
+                lm_events[t][1].record()
+            fr.fr_beam_step_lse(beam, lse[:rows], sl[:rows], 1 if t == 0 else K)
+        fr.fr_beam_finalize(beam, out_sids, out_scores, out_items)
+
+    for _ in range(args.warmup):
+        decode(hidden)
+    torch.cuda.synchronize()
+    for st in (fr.fr_lmhead_status(lm), fr.fr_beam_status(beam)):
+        if st != fr.FR_OK:
+            raise RuntimeError("lm_head decode failed: " + fr.fr_status_string(st))
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lm_ms = [[] for _ in range(D)]
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0.record()
+        for _ in range(args.steps):
+            decode(hidden)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier()
+        for _ in range(args.steps):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(D)]
+            decode(hidden, ev)
+            torch.cuda.synchronize()
+            for t in range(D):
+                lm_ms[t].append(ev[t][0].elapsed_time(ev[t][1]))
+    barrier()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dist, dev)
+    ms_per_decode = elapsed_ms / args.steps
+    value = job_throughput(world, B * K * D, args.steps, elapsed_ms)
+    flops = [2.0 * r * dh * V for r in rows_per_step]
+    lm_avg = [float(np.mean(x)) for x in lm_ms]
+    achieved = sum(flops) / (sum(lm_avg) / 1e3) / 1e12
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        peaks = json.load(f)
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "k_lmhead (+ k_lmhead_combine)",
+                "peak_source": "measured, sustained bf16 (cuBLAS)",
+                "flops_per_launch": sum(flops) / D, "ms_per_launch": sum(lm_avg) / D,
+                "timing": "CUDA events around fr_lmhead_run, second timed pass of the same decodes"}
+    per_step = [{"t": t, "rows": rows_per_step[t], "lmhead_ms": lm_avg[t],
+                 "tflops": flops[t] / (lm_avg[t] / 1e3) / 1e12} for t in range(D)]
+
+    e2e = None
+    if not args.no_e2e:
+        host = [h.cpu().pin_memory() for h in hidden]
+        dev_h = [torch.empty_like(h) for h in hidden]
+        h_sids = torch.empty((B, K, D), dtype=torch.int32, pin_memory=True)
+        h_scores = torch.empty((B, K), dtype=torch.float32, pin_memory=True)
+
+        def e2e_decode():
+            for t in range(D):
+                dev_h[t].copy_(host[t], non_blocking=True)
+            decode(dev_h)
+            h_sids.copy_(out_sids, non_blocking=True)
+            h_scores.copy_(out_scores, non_blocking=True)
+
+        e2e_decode()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.e2e_steps):
+            e2e_decode()
+        b_.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b_), world, dist, dev) / args.e2e_steps
+        e2e = {"value": world * B * K * D / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": sum(h.numel() * 2 for h in hidden),
+               "d2h_bytes_per_step": B * K * D * 4 + B * K * 4, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        n = 4
+        hh = hidden[1][0, :n].float().cpu().numpy()
+        ww = weight.float().cpu().numpy()
+        c0 = time.perf_counter()
+        oracle.lmhead_rows(hh, ww, w.sid_base, span)
+        per_row = (time.perf_counter() - c0) / n
+        rows_per_request = 1 + (D - 1) * K
+        cpu = {"value": K * D / (rows_per_request * per_row), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of "
+                         "request 0, %.2f s per row, scaled to one request's decode (%d rows: 1 at step 0, "
+                         "K afterwards); the selection's cost is negligible next to the rows"
+                         % (V, dh, n, per_row, rows_per_request)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
+            "config": {"workload": w.name, "path": "lm_head", "hidden_size": dh, "norm": args.norm,
+                       "temperature": args.temperature, "B_per_gpu": B, "K": K, "depth": D, "V": V,
+                       "codes_per_level": w.C, "catalog": w.n_items,
+                       "l2": "per step a distinct %.0f MB hidden-state buffer; the %.0f MB lm_head is re-read "
+                             "every step (larger than L2)" % (B * K * dh * 2 / 1e6, V * dh * 2 / 1e6),
+                       "step": "one full decode: depth x (fused lm_head + beam step) + finalize"},
+            "roofline": roofline, "per_step": per_step, "gpu_launches": args.steps * (4 * D + 2),
+            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    fr.fr_lmhead_destroy(lm)
+    fr.fr_beam_destroy(beam)
+    fr.fr_trie_destroy(trie)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.lmhead:
+        run_lmhead(args)
         return
     import torch
     import torch.distributed as dist
