@@ -981,7 +981,8 @@ __device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, 
 // gathers and the next step's candidate offsets.  All threads of the block
 // (blockDim.x >= K) call it.
 // Sorts the n (<= blockDim.x) distinct nonzero values sel[0..n) into
-// descending order: a bitonic network over P = max(32, next power of two >= n)
+// descending order.  Up to 256 values: by counting ranks.  More: a bitonic
+// network over P = max(32, next power of two >= n)
 // values held one per thread by threads 0..P-1, padded with 0 (below every
 // real value).  Compare-exchange partners closer than 32 are in the same warp
 // (shuffles); the farther ones exchange through shared memory, alternating
@@ -994,6 +995,28 @@ __device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
 
 __device__ void sort_desc_u64(unsigned long long* sel, unsigned long long* buf, int n) {
     const int tid = threadIdx.x;
+    if (n <= 256) {
+        // few values: each one's position is the number of values above it,
+        // counted over all n (every lane of a warp reads the same value, a
+        // broadcast, two values per 16-byte load)
+        unsigned long long v = 0ull;
+        int rank = 0;
+        if (tid < n) {
+            v = sel[tid];
+            const ulonglong2* s2 = reinterpret_cast<const ulonglong2*>(sel);
+            int j = 0;
+#pragma unroll 4
+            for (; j + 1 < n; j += 2) {
+                const ulonglong2 p = s2[j >> 1];
+                rank += (p.x > v) + (p.y > v);
+            }
+            if (j < n) rank += sel[j] > v;
+        }
+        __syncthreads();
+        if (tid < n) sel[rank] = v;
+        __syncthreads();
+        return;
+    }
     int P = 32;
     while (P < n) P <<= 1;
     if (tid < P) {  // whole warps: P is a multiple of 32
@@ -1096,7 +1119,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     griddep_launch_dependents();
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
-    __shared__ unsigned long long sel[FR_MAX_K];
+    __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_misc[4];
     __shared__ uint32_t red[64];
     const int b = blockIdx.x, tid = threadIdx.x;
@@ -1257,7 +1280,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     cg::cluster_group cl = cg::this_cluster();
     extern __shared__ __align__(16) uint32_t keys[];
     __shared__ __align__(16) int32_t hist[2][HBINS];
-    __shared__ unsigned long long sel[FR_MAX_K];
+    __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ uint32_t red[64];
     __shared__ int32_t s_misc[8];
@@ -1374,10 +1397,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
                 const int d = s_misc[1];
                 krem -= s_misc[2];
                 count_eq = s_misc[3];
-                if (tid == 0) {
-                    int before = 0;
-                    for (int r = 0; r < c; ++r) before += cl.map_shared_rank(h, r)[d];
-                    s_misc[4] = before;
+                if (tid < 32) {  // keys equal to the threshold digit in the slices before this one
+                    int before = tid < c ? cl.map_shared_rank(h, tid)[d] : 0;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+                    if (tid == 0) s_misc[4] = before;
                 }
                 prefix |= (uint32_t)d << shift;
                 lob = shift;
