@@ -52,25 +52,29 @@ namespace {
 #ifndef FR_NCW
 #define FR_NCW 16
 #endif
-#ifndef FR_STAGES
-#define FR_STAGES 6
-#endif
-#ifndef FR_STAGE_BYTES
-#define FR_STAGE_BYTES 32768
-#endif
 constexpr int NCW = FR_NCW;  // consumer warps: reduce the staged chunks
 constexpr int NFW = 2;       // finisher warps: lse, cross-CTA combine, candidate scores
 constexpr int PRODUCER_WARP = NCW;
 constexpr int FIRST_FINISHER_WARP = NCW + 1;
 constexpr int STREAM_THREADS = (NCW + 1 + NFW) * 32;
-constexpr int STAGES = FR_STAGES;
-constexpr int STAGE_BYTES = FR_STAGE_BYTES;
-constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-constexpr int VEC_PER_STAGE = STAGE_BYTES / 16;
-constexpr int VPL = VEC_PER_STAGE / (NCW * 32);  // 16-byte vectors per lane per chunk
+// The shared-memory ring of the streaming kernel, per element size (measured
+// on B200 over 3-7 stages of 32-64 KB: bf16 rows stream fastest through 4
+// stages of 48 KB, fp32 rows through 3 of 56 KB; larger chunks amortise the
+// per-chunk barrier work, and bf16 does twice the exponent work per byte).
+template <bool BF16>
+struct Ring {
+    static constexpr int STAGES = BF16 ? 4 : 3;
+    static constexpr int STAGE_BYTES = BF16 ? 49152 : 57344;
+    static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+    static constexpr int VEC_PER_STAGE = STAGE_BYTES / 16;
+    static constexpr int VPL = VEC_PER_STAGE / (NCW * 32);  // 16-byte vectors per lane per chunk
+    static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
+};
+constexpr int MAX_STAGES = 4;
+static_assert(Ring<true>::STAGES <= MAX_STAGES && Ring<false>::STAGES <= MAX_STAGES, "ring stages");
 constexpr int QCAP = 32;    // finished-segment jobs in flight per CTA
 constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
-static_assert(PSLOTS > 2 * STAGES, "partial slots must outnumber the segments in flight");
+static_assert(PSLOTS > 2 * MAX_STAGES, "partial slots must outnumber the segments in flight");
 constexpr int64_t GRAN = 1024;  // CTA ranges start at multiples of this many elements
 constexpr float L2E = 1.4426950408889634f;
 #ifndef FR_POLY_PAIRS
@@ -81,7 +85,6 @@ constexpr float L2E = 1.4426950408889634f;
 constexpr int POLY_PAIRS = FR_POLY_PAIRS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
-static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
 
 // Programmatic dependent launch (sm_90 and later).  The step kernels are
 // launched with programmatic stream serialization, so a kernel may be
@@ -100,8 +103,8 @@ struct Job {
 };
 
 struct SmemHdr {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     float2 part[PSLOTS][NCW];  // per-warp partials of a segment, slot = segment % PSLOTS
     int32_t segcnt[PSLOTS];
     Job jobs[QCAP];
@@ -228,7 +231,7 @@ template <int ELT>
 __device__ __forceinline__ Seg make_seg(const StreamArgs& a, const int32_t* row_start, int64_t r, int64_t bg,
                                         int64_t eg) {
     constexpr int64_t VE = 16 / ELT;          // elements per 16-byte vector
-    constexpr int64_t CE = STAGE_BYTES / ELT;  // elements per chunk
+    constexpr int64_t CE = Ring<ELT == 2>::STAGE_BYTES / ELT;  // elements per chunk
     Seg g;
     const int64_t rs = r * a.W;
     g.c0 = max(bg, rs) - rs;
@@ -340,7 +343,7 @@ __device__ __forceinline__ f32x2 exp2_poly_pair(f32x2 y) {
 
 // Exponent sum of this lane's VPL vectors against the reference point mref:
 // sum 2^(x*log2(e) - mref*log2(e)), in packed pairs.
-template <bool BF16, int POLY>
+template <bool BF16, int POLY, int VPL>
 __device__ __forceinline__ f32x2 lane_expsum(const uint4 (&q)[VPL], float mref) {
     const float nmL = (mref == -INFINITY) ? 0.f : -mref * L2E;
     const f32x2 c2 = pack2(nmL, nmL);
@@ -373,7 +376,7 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 }
 
 // Largest value of this lane's VPL vectors; NaN if any value is NaN.
-template <bool BF16>
+template <bool BF16, int VPL>
 __device__ __forceinline__ float lane_max(const uint4 (&q)[VPL]) {
     if constexpr (BF16) {
         __nv_bfloat162 h[4];
@@ -416,7 +419,7 @@ __device__ __forceinline__ float lane_max(const uint4 (&q)[VPL]) {
 // (on the MUFU alone, which keeps NaN and infinities intact).  The reference
 // is always one of the values seen, so the sum is at least 1 and a term that
 // underflows to zero is below 2^-126 of it.
-template <bool BF16>
+template <bool BF16, int VPL>
 __device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f32x2& s2) {
     float mref = m;
     if (mref == -INFINITY) mref = BF16 ? __uint_as_float(q[0].x << 16) : __uint_as_float(q[0].x);
@@ -569,6 +572,11 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
 template <bool BF16, bool LSE_ONLY>
 __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a) {
     constexpr int ELT = BF16 ? 2 : 4;
+    constexpr int STAGES = Ring<BF16>::STAGES;
+    constexpr int STAGE_BYTES = Ring<BF16>::STAGE_BYTES;
+    constexpr int RING_BYTES = Ring<BF16>::RING_BYTES;
+    constexpr int VEC_PER_STAGE = Ring<BF16>::VEC_PER_STAGE;
+    constexpr int VPL = Ring<BF16>::VPL;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* ring = smem;
     SmemHdr* hdr = reinterpret_cast<SmemHdr*>(smem + RING_BYTES);
@@ -803,6 +811,7 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
     const uint4* vec = reinterpret_cast<const uint4*>(sg.ptr + a0 * ELT);
     const uint32_t ninf = BF16 ? 0xFF80FF80u : 0xFF800000u;
     const uint4 ninf4 = make_uint4(ninf, ninf, ninf, ninf);
+    constexpr int VPL = 4;  // 16-byte vectors per lane per batch (2 KB per warp)
 
     float m = -INFINITY;
     f32x2 s2 = 0ull;
@@ -1579,15 +1588,17 @@ int small_grid(int64_t n) {
 
 }  // namespace
 
-size_t stream_smem_bytes(int32_t B) {
-    return (size_t)RING_BYTES + sizeof(SmemHdr) + sizeof(int32_t) * (size_t)(B + 1);
+size_t stream_smem_bytes(int32_t B, bool bf16) {
+    return (size_t)(bf16 ? Ring<true>::RING_BYTES : Ring<false>::RING_BYTES) + sizeof(SmemHdr) +
+           sizeof(int32_t) * (size_t)(B + 1);
 }
 
 cudaError_t stream_kernel_setup() {
-    const int max_bytes = (int)stream_smem_bytes(FR_MAX_B);
-    cudaError_t e = cudaFuncSetAttribute(k_stream<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)stream_smem_bytes(FR_MAX_B, true));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_stream<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    return cudaFuncSetAttribute(k_stream<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)stream_smem_bytes(FR_MAX_B, false));
 }
 
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t, const void* logits,
@@ -1631,7 +1642,7 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
         return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_rows_short<true>, a)
                                    : cudaLaunchKernelEx(&L.cfg, k_rows_short<false>, a);
     }
-    StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B), s);
+    StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B, sh.dtype == FR_BF16), s);
     return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true, false>, a)
                                : cudaLaunchKernelEx(&L.cfg, k_stream<false, false>, a);
 }
@@ -1677,10 +1688,9 @@ cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const T
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
                            const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
                            cudaStream_t s) {
-    const int max_bytes = (int)stream_smem_bytes(1);
-    cudaError_t e = cudaFuncSetAttribute(k_stream<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_stream<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
+    const int max_bytes = (int)stream_smem_bytes(1, dtype == FR_BF16);
+    cudaError_t e = cudaFuncSetAttribute(dtype == FR_BF16 ? k_stream<true, true> : k_stream<false, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
     if (e != cudaSuccess) return e;
     StreamArgs a{};
     a.logits = static_cast<const char*>(logits);

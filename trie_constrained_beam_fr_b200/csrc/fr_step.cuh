@@ -37,8 +37,9 @@ struct StepShape {
 // `bound` candidates (0 = the single-CTA kernel).
 int select_cluster_size(int32_t B, int64_t bound, int32_t sms);
 
-// Streaming kernel: dynamic shared memory it needs for B requests.
-size_t stream_smem_bytes(int32_t B);
+// Streaming kernel: dynamic shared memory it needs for B requests (bf16 or
+// fp32 rows: the ring differs).
+size_t stream_smem_bytes(int32_t B, bool bf16);
 cudaError_t stream_kernel_setup();  // raises the kernel's shared-memory limit
 
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
