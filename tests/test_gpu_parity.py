@@ -45,6 +45,13 @@ SMALL = {
                            dtype="f32", seed=7, catalog_seed=7),
     "skewed_small": W("skewed_small", B=2, K=128, depth=3, C=256, V=5000, sid_base=1000, n_items=30000,
                       dtype="f32", seed=8, catalog_seed=8, zipf_levels=2),
+    # the largest request count the library takes (its row table fills the
+    # streaming kernel's shared memory beside the ring); rows of 36 KB
+    "max_requests": W("max_requests", B=4096, K=2, depth=2, C=16, V=9000, sid_base=100, n_items=200,
+                      dtype="f32", seed=13, catalog_seed=13),
+    # a deep trie: 12 levels of 4 codes
+    "deep": W("deep", B=2, K=16, depth=12, C=4, V=200, sid_base=100, n_items=5000, dtype="bf16", seed=14,
+              catalog_seed=14),
     # K x max fan-out = 1024 x 1024 candidates: beyond what a 16-CTA cluster
     # holds in shared memory, so the selection reads the candidates from L2
     "k1024_wide_fanout": W("k1024_wide_fanout", B=2, K=1024, depth=2, C=1024, V=2100, sid_base=30,
