@@ -12,10 +12,11 @@
 //            space of all live rows (request-major) is cut into equal,
 //            1024-element-aligned ranges, one per CTA, so every CTA streams
 //            the same number of bytes whatever the row count.  Inside a CTA
-//            one producer lane moves 32 KB chunks from HBM into a 6-stage
-//            shared-memory ring with 1-D bulk async copies completing on
-//            mbarriers; 16 consumer warps each reduce a 2 KB slice of every
-//            chunk (running reference + scaled exp2 sum per lane).  At the end of a
+//            one producer lane moves chunks from HBM into a shared-memory
+//            ring (bf16: 4 stages of 48 KB; fp32: 3 of 56 KB) with 1-D bulk
+//            async copies completing on mbarriers; 16 consumer warps each
+//            reduce a lane-interleaved slice of every chunk (running
+//            reference + scaled exp2 sum per lane).  At the end of a
 //            row segment the last consumer warp to arrive combines the 16
 //            warp partials in a fixed order and finishes the row; a row split
 //            across CTAs is finished by the last CTA to arrive (atomic
@@ -25,8 +26,9 @@
 //  k_select  per request: exact top-K of all its candidates under the strict
 //            order (score desc, slot asc) -- slot order is (parent slot,
 //            token) order -- by radix selection of order-preserving 32-bit
-//            keys (12-bit digits after skipping the bits all keys share),
-//            then a bitonic sort of the K winners on (key, ~slot); then the
+//            keys (12-bit digits after skipping the bits all keys share;
+//            a thread-block cluster per request when a request has many
+//            candidates), then a sort of the K winners on (key, ~slot); then the
 //            reorder gathers: backpointer, token, trie node, score, prefix and
 //            KV slot of every survivor, and the next step's candidate offsets.
 //
