@@ -97,7 +97,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
         // step t: live beams (1 at the root, then at most K) times the level's fan-out
         const int64_t bound = (int64_t)(t == 0 ? 1 : K) * std::max(1, trie->level_fanout[t]);
         bm->shape.sel_bound[t] = bound;
-        bm->shape.sel_cluster[t] = fr::select_cluster_size(B, bound, sms);
+        bm->shape.sel_cluster[t] = fr::select_cluster_size(B, K, bound, sms);
     }
     const size_t bk = (size_t)B * K;
     const int64_t cand_stride = (int64_t)K * std::max(1, trie->max_fanout);

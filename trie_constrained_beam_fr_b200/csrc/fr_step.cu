@@ -944,7 +944,8 @@ struct SelectArgs {
     int32_t* parent_out;
     int32_t* token_out;
     int32_t* err;
-    int32_t key_cap;  // cluster select: keys each CTA's shared memory holds
+    int32_t key_cap;   // cluster select: keys each CTA's shared memory holds
+    int32_t pool_cap;  // cluster select: values the leader's pool holds
 };
 
 __device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t* out_or) {
@@ -1125,56 +1126,72 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
 }
 
 
-__global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
-    griddep_wait();
-    griddep_launch_dependents();
-    __shared__ int32_t s_off[FR_MAX_K + 1];
-    __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
-    __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
-    __shared__ int32_t s_misc[4];
-    __shared__ uint32_t red[64];
-    const int b = blockIdx.x, tid = threadIdx.x;
-    const int K = a.K;
-    const int live = min(max(a.cur.live[b], 0), K);
-    for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
-    __syncthreads();
-    int n = s_off[live];
-    if (n < 0 || (int64_t)n > a.cand_stride) {
-        if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
-        n = 0;
+// Candidate values for the selection: val(i) = (key << 32) | low, with key an
+// order-preserving image of the candidate's score (or sampling key) and low =
+// ~slot, so that larger values come first in the step's total order (key
+// descending, slot ascending) and index order is slot order.
+struct GlobalCands {  // the request's candidates in global memory, slot i at cb[i]
+    const float* cb;
+    __device__ __forceinline__ uint32_t key(int i) const { return float_to_key(__ldg(cb + i)); }
+    __device__ __forceinline__ unsigned long long val(int i) const {
+        return ((unsigned long long)key(i) << 32) | (0xFFFFFFFFu - (uint32_t)i);
     }
-    const int Kp = min(K, n);
-    const float* cb = a.rank + (int64_t)b * a.cand_stride;
+};
+struct SmemKeys {  // a contiguous slice of them, as keys in shared memory, slot base + i at keys[i]
+    const uint32_t* keys;
+    uint32_t base;
+    __device__ __forceinline__ uint32_t key(int i) const { return keys[i]; }
+    __device__ __forceinline__ unsigned long long val(int i) const {
+        return ((unsigned long long)keys[i] << 32) | (0xFFFFFFFFu - (base + (uint32_t)i));
+    }
+};
+struct PoolVals {  // values already formed, in slot order
+    const unsigned long long* pool;
+    __device__ __forceinline__ uint32_t key(int i) const { return (uint32_t)(pool[i] >> 32); }
+    __device__ __forceinline__ unsigned long long val(int i) const { return pool[i]; }
+};
 
-    if (Kp > 0 && Kp == n) {
-        // every candidate survives: no threshold to find
-        for (int i = tid; i < n; i += SEL_THREADS)
-            sel[i] = ((unsigned long long)float_to_key(__ldg(cb + i)) << 32) | (0xFFFFFFFFu - (uint32_t)i);
-        __syncthreads();
-    } else if (Kp > 0) {
+// Exact top-Kp (Kp <= n, Kp <= FR_MAX_K) of the n values under the total
+// order: the Kp winners' values go to out[0..Kp); the return value is how
+// many were written (Kp unless something is inconsistent).  The Kp-th key T
+// is found by radix selection on the keys (12-bit digits after skipping the
+// bits every key shares); the winners are every key > T and the lowest-index
+// keys == T.  ORDERED: they are written in index (slot) order -- each warp
+// owns a contiguous block of indices and counts its keys above and at T
+// (ballots), one scan over the warps gives each warp its output offset, and a
+// second sweep writes.  Otherwise in any order, in one sweep (atomic
+// positions; the keys equal to T are taken in index order, by block scans,
+// only when not all of them win).  All threads of the block call it; scratch:
+// hist [HBINS], red [64], s_misc [8].
+template <bool ORDERED, class Vals>
+__device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* out, int32_t* hist, uint32_t* red,
+                          int32_t* s_misc) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (Kp <= 0 || n <= 0) return 0;
+    uint32_t T = 0u;
+    int eq_needed = n;  // Kp == n: every value wins (all keys are >= 0)
+    int count_eq = n;   // keys equal to T (an upper bound when every value wins)
+    if (Kp < n) {
         uint32_t va = 0xFFFFFFFFu, vo = 0u;
         int i0 = tid;
         for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-            float x[8];
+            uint32_t k8[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+            for (int u = 0; u < 8; ++u) k8[u] = vals.key(i0 + u * SEL_THREADS);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const uint32_t k = float_to_key(x[u]);
-                va &= k;
-                vo |= k;
+                va &= k8[u];
+                vo |= k8[u];
             }
         }
         for (int i = i0; i < n; i += SEL_THREADS) {
-            const uint32_t k = float_to_key(__ldg(cb + i));
+            const uint32_t k = vals.key(i);
             va &= k;
             vo |= k;
         }
         uint32_t VO;
         const uint32_t VA = block_and_or(va, vo, red, &VO);
         const uint32_t diff = VA ^ VO;
-        uint32_t T;
-        int eq_needed, count_eq;
         if (diff == 0u) {
             T = VA;
             eq_needed = Kp;
@@ -1183,7 +1200,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
             int lo = 32 - __clz(diff);  // bits >= lo are the same in every key
             uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
             int krem = Kp;
-            count_eq = 0;
             while (lo > 0) {
                 const int width = min(HBITS, lo);
                 const int shift = lo - width;
@@ -1191,19 +1207,17 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
                 for (int i = tid; i < HBINS; i += SEL_THREADS) hist[i] = 0;
                 __syncthreads();
                 const uint64_t want = (uint64_t)prefix >> lo;
-                int i0 = tid;
-                for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-                    float x[8];
+                int j0 = tid;
+                for (; j0 + 7 * SEL_THREADS < n; j0 += 8 * SEL_THREADS) {
+                    uint32_t k8[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+                    for (int u = 0; u < 8; ++u) k8[u] = vals.key(j0 + u * SEL_THREADS);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t k = float_to_key(x[u]);
-                        if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
-                    }
+                    for (int u = 0; u < 8; ++u)
+                        if (((uint64_t)k8[u] >> lo) == want) atomicAdd(&hist[(k8[u] >> shift) & dmask], 1);
                 }
-                for (int i = i0; i < n; i += SEL_THREADS) {
-                    const uint32_t k = float_to_key(__ldg(cb + i));
+                for (int i = j0; i < n; i += SEL_THREADS) {
+                    const uint32_t k = vals.key(i);
                     if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
                 }
                 __syncthreads();
@@ -1226,76 +1240,183 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
                     cum += h4[q];
                 }
                 __syncthreads();
-                const int d = s_misc[0];
                 krem -= s_misc[1];
                 count_eq = s_misc[2];
-                prefix |= (uint32_t)d << shift;
+                prefix |= (uint32_t)s_misc[0] << shift;
                 lo = shift;
                 __syncthreads();
             }
             T = prefix;
             eq_needed = krem;
         }
-        // collect the Kp winners: every key > T and the eq_needed lowest slots with key == T
+    }
+    if constexpr (!ORDERED) {
         if (tid == 0) s_misc[3] = 0;
         __syncthreads();
-        if (eq_needed >= count_eq) {
-            for (int i = tid; i < n; i += SEL_THREADS) {
-                const uint32_t k = float_to_key(__ldg(cb + i));
-                if (k >= T) {
+        if (eq_needed >= count_eq) {  // every key >= T wins
+            int i0 = tid;
+            for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
+                unsigned long long v8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v8[u] = vals.val(i0 + u * SEL_THREADS);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if ((uint32_t)(v8[u] >> 32) >= T) {
+                        const int p = atomicAdd(&s_misc[3], 1);
+                        if (p < Kp) out[p] = v8[u];
+                    }
+            }
+            for (int i = i0; i < n; i += SEL_THREADS) {
+                const unsigned long long v = vals.val(i);
+                if ((uint32_t)(v >> 32) >= T) {
                     const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < FR_MAX_K) sel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
+                    if (p < Kp) out[p] = v;
                 }
             }
-        } else {
+        } else {  // the keys equal to T straddle the boundary: take them in index order
             int run_eq = 0;
             for (int base = 0; base < n; base += SEL_THREADS) {
                 const int i = base + tid;
-                const uint32_t k = i < n ? float_to_key(__ldg(cb + i)) : 0u;
+                const unsigned long long v = i < n ? vals.val(i) : 0ull;
+                const uint32_t k = (uint32_t)(v >> 32);
                 const bool gt = i < n && k > T;
                 const bool eq = i < n && k == T;
                 int tot;
                 const int r = block_excl_scan(eq ? 1 : 0, &tot);
                 if (gt || (eq && run_eq + r < eq_needed)) {
                     const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < FR_MAX_K) sel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
+                    if (p < Kp) out[p] = v;
                 }
                 run_eq += tot;
             }
         }
         __syncthreads();
-        if (tid == 0 && s_misc[3] != Kp) set_error(a.err, FR_ERR_DEVICE);
+        return s_misc[3];
     }
+    // collect in index order
+    constexpr int NW = SEL_THREADS / 32;
+    const int per = (((n + NW - 1) / NW) + 31) & ~31;
+    const int beg = min(n, warp * per), end = min(n, beg + per);
+    constexpr int CB = 8;  // 32-wide rows per batch: CB independent loads in flight per lane
+    int cgt = 0, ceq = 0;
+    for (int j = beg; j < end; j += 32 * CB) {
+        uint32_t k8[CB];
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const int i = j + u * 32 + lane;
+            k8[u] = i < end ? vals.key(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const bool in = j + u * 32 + lane < end;
+            cgt += __popc(__ballot_sync(0xffffffffu, in && k8[u] > T));
+            ceq += __popc(__ballot_sync(0xffffffffu, in && k8[u] == T));
+        }
+    }
+    if (lane == 0) {
+        red[warp] = (uint32_t)cgt;
+        red[NW + warp] = (uint32_t)ceq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int g = lane < NW ? (int)red[lane] : 0, e = lane < NW ? (int)red[NW + lane] : 0;
+        const int gi = warp_incl_scan(g), ei = warp_incl_scan(e);
+        if (lane < NW) {
+            red[lane] = (uint32_t)(gi - g);
+            red[NW + lane] = (uint32_t)(ei - e);
+        }
+        if (lane == 31) {
+            s_misc[6] = gi;
+            s_misc[7] = ei;
+        }
+    }
+    __syncthreads();
+    int gbase = (int)red[warp], ebase = (int)red[NW + warp];
+    const int total = s_misc[6] + min(s_misc[7], eq_needed);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j = beg; j < end; j += 32 * CB) {
+        unsigned long long v8[CB];
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const int i = j + u * 32 + lane;
+            v8[u] = i < end ? vals.val(i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const bool in = j + u * 32 + lane < end;
+            const uint32_t k = (uint32_t)(v8[u] >> 32);
+            const bool g = in && k > T, e = in && k == T;
+            const unsigned bg = __ballot_sync(0xffffffffu, g), be = __ballot_sync(0xffffffffu, e);
+            const int gb = gbase + __popc(bg & lt), eb = ebase + __popc(be & lt);
+            int pos = -1;
+            if (g) pos = gb + min(eb, eq_needed);
+            else if (e && eb < eq_needed) pos = gb + eb;
+            if (pos >= 0 && pos < Kp) out[pos] = v8[u];
+            gbase += __popc(bg);
+            ebase += __popc(be);
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ int32_t s_off[FR_MAX_K + 1];
+    __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
+    __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
+    __shared__ int32_t s_misc[8];
+    __shared__ uint32_t red[64];
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int K = a.K;
+    const int live = min(max(a.cur.live[b], 0), K);
+    for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
+    __syncthreads();
+    int n = s_off[live];
+    if (n < 0 || (int64_t)n > a.cand_stride) {
+        if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
+        n = 0;
+    }
+    const int Kp = min(K, n);
+    const int got = block_topk<false>(GlobalCands{a.rank + (int64_t)b * a.cand_stride}, n, Kp, sel, hist, red, s_misc);
+    if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
     select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
 // ---------------------------------------------------------------------------
 // Selection with one thread-block cluster per request.  Each CTA of the
-// cluster holds a contiguous slice of the request's candidates in shared
-// memory as order-preserving keys, loaded once; the bits shared by every key
-// are skipped (cluster-wide AND/OR), and each 12-bit radix pass histograms the
-// slices locally, after which every CTA reads all peers' histograms through
-// distributed shared memory and derives the same threshold digit.  Winners go
-// straight into the leader CTA's array (DSMEM atomics); keys equal to the
-// threshold are taken in slot order (slices are contiguous in slot order, so
-// each CTA starts from the count of equal keys in the slices before it).  The
-// leader sorts and emits.  Every CTA runs the same sequence of cluster
-// barriers: their number depends only on cluster-wide values.
+// cluster loads a contiguous slice of the request's candidates into shared
+// memory as keys and selects the slice's exact top-K with block barriers only
+// (block_topk); the union of the slices' top-Ks holds the request's top-K.
+// After one cluster barrier the leader CTA copies the CTAs' winner lists
+// (each in slot order, the slices in slot order) through distributed shared
+// memory into a pool in its own key area, a second cluster barrier releases
+// the other CTAs, and the leader selects the top-K of the pool, sorts it and
+// emits.  Every CTA runs the same two cluster barriers.
 
 namespace cg = cooperative_groups;
 constexpr int CSEL_MAXKEYS = 40960;  // keys per CTA (160 KB of shared memory)
+
+// Dynamic shared memory of the cluster selection: a CTA's keys, and in the
+// leader later the pool of up to cs * min(K, keys per CTA) values.
+size_t csel_smem_bytes(int64_t key_cap, int cs, int K) {
+    const int64_t pool = (int64_t)cs * (K < key_cap ? K : key_cap);
+    const int64_t kb = key_cap * (int64_t)sizeof(uint32_t), pb = pool * (int64_t)sizeof(unsigned long long);
+    return (size_t)(kb > pb ? kb : pb);
+}
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectArgs a) {
     griddep_wait();
     griddep_launch_dependents();
     cg::cluster_group cl = cg::this_cluster();
-    extern __shared__ __align__(16) uint32_t keys[];
-    __shared__ __align__(16) int32_t hist[2][HBINS];
+    extern __shared__ __align__(16) uint32_t keys[];  // this CTA's keys; in the leader, then the pool
+    __shared__ __align__(16) int32_t hist[HBINS];    // also the sort's scratch
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ uint32_t red[64];
     __shared__ int32_t s_misc[8];
-    __shared__ uint32_t s_ao[2];
+    __shared__ int32_t s_cnt;
     const int CS = (int)cl.num_blocks();
     const int c = (int)cl.block_rank();
     const int b = blockIdx.x / CS;
@@ -1312,153 +1433,44 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     const int S = (n + CS - 1) / CS;
     const int lo = min(n, c * S), hi = min(n, lo + S);
     const int cnt = hi - lo;
-    if (c == 0) {
+    if (c == 0)
         for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = off_row[i];
-        if (tid == 0) s_misc[0] = 0;  // the leader's winner count
-    }
     const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;
-    uint32_t va = 0xFFFFFFFFu, vo = 0u;
     int i0 = tid;
     for (; i0 + 7 * SEL_THREADS < cnt; i0 += 8 * SEL_THREADS) {
         float x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const uint32_t k = float_to_key(x[u]);
-            keys[i0 + u * SEL_THREADS] = k;
-            va &= k;
-            vo |= k;
-        }
+        for (int u = 0; u < 8; ++u) keys[i0 + u * SEL_THREADS] = float_to_key(x[u]);
     }
-    for (int i = i0; i < cnt; i += SEL_THREADS) {
-        const uint32_t k = float_to_key(__ldg(cb + i));
-        keys[i] = k;
-        va &= k;
-        vo |= k;
-    }
-    uint32_t VO;
-    const uint32_t VA = block_and_or(va, vo, red, &VO);
+    for (int i = i0; i < cnt; i += SEL_THREADS) keys[i] = float_to_key(__ldg(cb + i));
+    __syncthreads();
+    const int kc = min(Kp, cnt);
+    const int nloc = block_topk<true>(SmemKeys{keys, (uint32_t)lo}, cnt, kc, sel, hist, red, s_misc);
     if (tid == 0) {
-        s_ao[0] = VA;
-        s_ao[1] = VO;
+        s_cnt = nloc > 0 ? nloc : 0;
+        if (nloc != kc) set_error(a.err, FR_ERR_DEVICE);
     }
-    cl.sync();
-    uint32_t GA = 0xFFFFFFFFu, GO = 0u;
-    for (int r = 0; r < CS; ++r) {
-        const uint32_t* p = cl.map_shared_rank(s_ao, r);
-        GA &= p[0];
-        GO |= p[1];
-    }
-
-    uint32_t T = 0u;
-    int eq_needed = 0, count_eq = 0, eq_before = 0;
-    if (Kp > 0) {
-        const uint32_t diff = GA ^ GO;
-        if (Kp == n) {
-            // every candidate survives: every key is >= 0 and all are taken
-            T = 0u;
-            eq_needed = count_eq = n;
-        } else if (diff == 0u) {
-            T = GA;
-            eq_needed = Kp;
-            count_eq = n;
-            eq_before = lo;
-        } else {
-            int lob = 32 - __clz(diff);
-            uint32_t prefix = (lob == 32) ? 0u : (GA & (0xFFFFFFFFu << lob));
-            int krem = Kp;
-            int pass = 0;
-            while (lob > 0) {
-                const int width = min(HBITS, lob);
-                const int shift = lob - width;
-                const uint32_t dmask = (1u << width) - 1u;
-                int32_t* h = hist[pass & 1];
-                for (int i = tid; i < HBINS; i += SEL_THREADS) h[i] = 0;
-                __syncthreads();
-                const uint64_t want = (uint64_t)prefix >> lob;
-                for (int i = tid; i < cnt; i += SEL_THREADS) {
-                    const uint32_t k = keys[i];
-                    if (((uint64_t)k >> lob) == want) atomicAdd(&h[(k >> shift) & dmask], 1);
-                }
-                __syncthreads();
-                cl.sync();
-                int g4[4] = {0, 0, 0, 0};
-                for (int r = 0; r < CS; ++r) {
-                    const int4 v = *reinterpret_cast<const int4*>(cl.map_shared_rank(h, r) + tid * 4);
-                    g4[0] += v.x;
-                    g4[1] += v.y;
-                    g4[2] += v.z;
-                    g4[3] += v.w;
-                }
-                const int tsum = g4[0] + g4[1] + g4[2] + g4[3];
-                int tot;
-                const int excl = block_excl_scan(tsum, &tot);
-                int cum = tot - excl - tsum;  // keys in the bins above this thread's
-#pragma unroll
-                for (int q = 3; q >= 0; --q) {
-                    if (cum < krem && cum + g4[q] >= krem) {
-                        s_misc[1] = tid * 4 + q;
-                        s_misc[2] = cum;
-                        s_misc[3] = g4[q];
-                    }
-                    cum += g4[q];
-                }
-                __syncthreads();
-                const int d = s_misc[1];
-                krem -= s_misc[2];
-                count_eq = s_misc[3];
-                if (tid < 32) {  // keys equal to the threshold digit in the slices before this one
-                    int before = tid < c ? cl.map_shared_rank(h, tid)[d] : 0;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
-                    if (tid == 0) s_misc[4] = before;
-                }
-                prefix |= (uint32_t)d << shift;
-                lob = shift;
-                ++pass;
-                __syncthreads();
-                eq_before = s_misc[4];
+    cl.sync();  // every slice's winners are in its CTA's sel
+    unsigned long long* pool = reinterpret_cast<unsigned long long*>(keys);
+    int P = 0;
+    if (c == 0) {
+        for (int r = 0; r < CS; ++r) {
+            const int cr = *cl.map_shared_rank(&s_cnt, r);
+            if ((int64_t)P + cr > a.pool_cap) {  // cannot happen: the pool holds CS * min(K, keys per CTA)
+                if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
+                break;
             }
-            T = prefix;
-            eq_needed = krem;
+            const unsigned long long* src = cl.map_shared_rank(sel, r);
+            for (int i = tid; i < cr; i += SEL_THREADS) pool[P + i] = src[i];
+            P += cr;
         }
     }
-    // collect: every key > T, and the keys == T whose slot-order rank among
-    // the equal keys is below eq_needed
-    unsigned long long* lsel = cl.map_shared_rank(sel, 0);
-    int32_t* lcnt = cl.map_shared_rank(&s_misc[0], 0);
-    if (Kp > 0) {
-        const bool all_eq = eq_needed >= count_eq;
-        const bool no_eq = !all_eq && eq_before >= eq_needed;
-        if (all_eq || no_eq) {
-            for (int i = tid; i < cnt; i += SEL_THREADS) {
-                const uint32_t k = keys[i];
-                if (k > T || (all_eq && k == T)) {
-                    const int p = atomicAdd(lcnt, 1);
-                    if (p < FR_MAX_K) lsel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i));
-                }
-            }
-        } else {
-            int run = eq_before;
-            for (int base = 0; base < cnt; base += SEL_THREADS) {
-                const int i = base + tid;
-                const uint32_t k = i < cnt ? keys[i] : 0u;
-                const bool gt = i < cnt && k > T;
-                const bool eq = i < cnt && k == T;
-                int tot;
-                const int r = block_excl_scan(eq ? 1 : 0, &tot);
-                if (gt || (eq && run + r < eq_needed)) {
-                    const int p = atomicAdd(lcnt, 1);
-                    if (p < FR_MAX_K) lsel[p] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i));
-                }
-                run += tot;
-            }
-        }
-    }
-    cl.sync();
+    cl.sync();  // the leader has read every list: the other CTAs may leave
     if (c != 0) return;
-    if (tid == 0 && s_misc[0] != Kp) set_error(a.err, FR_ERR_DEVICE);
+    const int got = block_topk<false>(PoolVals{pool}, P, min(Kp, P), sel, hist, red, s_misc);
+    if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
     select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
@@ -1737,17 +1749,19 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
         return cudaLaunchKernelEx(&L.cfg, k_select, a);
     }
     a.key_cap = (int32_t)((sh.sel_bound[t] + cs - 1) / cs);
-    StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, (size_t)a.key_cap * sizeof(uint32_t), s, (unsigned)cs);
+    a.pool_cap = cs * (sh.K < a.key_cap ? sh.K : a.key_cap);
+    StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, csel_smem_bytes(a.key_cap, cs, sh.K), s, (unsigned)cs);
     return cudaLaunchKernelEx(&L.cfg, k_select_cluster, a);
 }
 
-int select_cluster_size(int32_t B, int64_t bound, int32_t sms) {
+int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {
     // Few candidates: one CTA per request is quickest (no cluster barriers).
-    // Very many: they do not fit a small cluster's shared memory; one CTA per
-    // request reads them from L2.  In between, a cluster of up to 4 CTAs per
-    // request, as long as every request's cluster runs in the same wave.
+    // Very many: they do not fit a cluster's shared memory; one CTA per
+    // request reads them from L2.  In between, a cluster of up to 8 CTAs per
+    // request (enough to hold the keys; more while the GPU has idle SMs), as
+    // long as every request's cluster runs in the same wave.
     constexpr int64_t SMALL_BOUND = 8192;
-    constexpr int MAX_CS = 4;
+    constexpr int MAX_CS = 8;  // the portable cluster size
     if (bound <= SMALL_BOUND) return 0;
     int need = 1;
     while ((bound + need - 1) / need > CSEL_MAXKEYS) need <<= 1;
@@ -1757,14 +1771,14 @@ int select_cluster_size(int32_t B, int64_t bound, int32_t sms) {
     const int cs = need > fill ? need : fill;
     if (cs < 2 || (int64_t)B * cs > sms) return 0;
     if (cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CSEL_MAXKEYS * (int)sizeof(uint32_t)) != cudaSuccess) {
+                             (int)csel_smem_bytes(CSEL_MAXKEYS, 8, FR_MAX_K)) != cudaSuccess) {
         (void)cudaGetLastError();
         return 0;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(B * cs));
     cfg.blockDim = dim3(SEL_THREADS);
-    cfg.dynamicSmemBytes = (size_t)((bound + cs - 1) / cs) * sizeof(uint32_t);
+    cfg.dynamicSmemBytes = csel_smem_bytes((bound + cs - 1) / cs, cs, K);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;

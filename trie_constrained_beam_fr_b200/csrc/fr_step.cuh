@@ -35,7 +35,7 @@ struct StepShape {
 
 // Cluster size of the selection for a step whose requests have at most
 // `bound` candidates (0 = the single-CTA kernel).
-int select_cluster_size(int32_t B, int64_t bound, int32_t sms);
+int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms);
 
 // Streaming kernel: dynamic shared memory it needs for B requests (bf16 or
 // fp32 rows: the ring differs).
