@@ -17,9 +17,12 @@ pytestmark = pytest.mark.gpu
 
 W = synth.Workload
 # Rows whose streamed window is at most 16 KB take the warp-per-row kernel
-# (tiny, ragged_bf16, k1024, greedy, k_exceeds_catalog, k1024_wide_fanout);
-# longer rows take the persistent streaming kernel (ragged_wide_bf16,
-# mid_bf16, mid_f32_deep, full_vocab_few_rows, skewed_small).
+# (tiny, ragged_bf16, k1024, greedy, k_exceeds_catalog, k1024_wide_fanout,
+# cluster2, cluster4, deep); longer rows take the persistent streaming kernel
+# (ragged_wide_bf16, mid_bf16, mid_f32_deep, full_vocab_few_rows,
+# skewed_small, max_requests).  Selections over more than 16,384 candidates
+# per request run in thread-block clusters: k1024 and skewed_small (8 CTAs),
+# cluster2 (2), cluster4 (4).
 SMALL = {
     # the tiny workload itself
     "tiny": synth.WORKLOADS["tiny"],
@@ -49,6 +52,12 @@ SMALL = {
     # streaming kernel's shared memory beside the ring); rows of 36 KB
     "max_requests": W("max_requests", B=4096, K=2, depth=2, C=16, V=9000, sid_base=100, n_items=200,
                       dtype="f32", seed=13, catalog_seed=13),
+    # step 1 selects over ~25,000 candidates per request in a cluster of 2
+    # (40 requests) and of 4 (20 requests) CTAs per request
+    "cluster2": W("cluster2", B=40, K=256, depth=2, C=256, V=2000, sid_base=500, n_items=20000, dtype="bf16",
+                  seed=15, catalog_seed=15),
+    "cluster4": W("cluster4", B=20, K=256, depth=2, C=256, V=2000, sid_base=500, n_items=20000, dtype="bf16",
+                  seed=15, catalog_seed=15),
     # a deep trie: 12 levels of 4 codes
     "deep": W("deep", B=2, K=16, depth=12, C=4, V=200, sid_base=100, n_items=5000, dtype="bf16", seed=14,
               catalog_seed=14),

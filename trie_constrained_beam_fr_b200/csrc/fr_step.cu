@@ -1760,7 +1760,7 @@ int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {
     // request reads them from L2.  In between, a cluster of up to 8 CTAs per
     // request (enough to hold the keys; more while the GPU has idle SMs), as
     // long as every request's cluster runs in the same wave.
-    constexpr int64_t SMALL_BOUND = 8192;
+    constexpr int64_t SMALL_BOUND = 16384;  // measured: one CTA is quicker up to here
     constexpr int MAX_CS = 8;  // the portable cluster size
     if (bound <= SMALL_BOUND) return 0;
     int need = 1;
