@@ -192,7 +192,10 @@ fr_status fr_beam_finalize(fr_beam* beam, int32_t* sids_dev, float* scores_dev, 
 /* init allocates the partials for up to max_rows rows; run is stream-ordered */
 /* and asynchronous; status synchronises and returns the sticky device status */
 /* (FR_ERR_NAN_LOGIT for a non-finite row, FR_ERR_DEVICE on an internal       */
-/* timeout). */
+/* timeout).  The kernel takes one CTA per SM with ~198 KB of shared memory   */
+/* and all 512 tensor-memory columns of the SM while it runs, so kernels of   */
+/* the caller that also allocate tensor memory should not run concurrently    */
+/* with it on other streams (their allocation would wait for it). */
 typedef struct fr_lmhead fr_lmhead;
 fr_status fr_lmhead_init(const void* weight_dev, int64_t ldw, int32_t V, int32_t d, int32_t max_rows,
                          int32_t sid_base, int32_t sid_span, fr_lmhead** out);
