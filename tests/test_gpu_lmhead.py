@@ -97,3 +97,34 @@ def test_lmhead_rejects_bad_arguments():
             fr.fr_lmhead_run(lm, flat[1:].view(8, 64), lse, sl)  # base not 16-byte aligned
     finally:
         fr.fr_lmhead_destroy(lm)
+
+
+@pytest.mark.slow
+def test_lmhead_full_size_sampled_rows():
+    """The serving shape in the launch configuration the benchmark times
+    (8,192 rows x d 2,048 x V 151,936, SID range at 131,072): every row's
+    log-sum-exp is finite, and sampled rows (first, last, one per tile
+    boundary) match the oracle's rows in double within the accumulation
+    bound."""
+    rows, d, V, sb, span = 8192, 2048, 151936, 131072, 768
+    g = torch.Generator().manual_seed(11)
+    Wd = (torch.randn(V, d, generator=g) / d ** 0.5).to(torch.bfloat16).cuda()
+    hd = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    lm = fr.fr_lmhead_init(Wd, max_rows=rows, sid_base=sb, sid_span=span)
+    try:
+        lse = torch.empty(rows, device="cuda")
+        sl = torch.empty(rows, span, device="cuda")
+        fr.fr_lmhead_run(lm, hd, lse, sl)
+        assert fr.fr_lmhead_status(lm) == fr.FR_OK
+        lse_all = lse.cpu().numpy()
+        sl_all = sl.cpu().numpy()
+    finally:
+        fr.fr_lmhead_destroy(lm)
+    assert np.all(np.isfinite(lse_all))
+    pick = [0, 127, 128, 4095, 8191]
+    h = hd[pick].float().cpu().numpy()
+    W = Wd.float().cpu().numpy()
+    lse_ref, sl_ref = oracle.lmhead_rows(h, W, sb, span)
+    bound = d * 2.0 ** -23 * (np.abs(h).astype(np.float64) @ np.abs(W).astype(np.float64).T)
+    assert np.all(np.abs(lse_all[pick] - lse_ref) <= bound.max(axis=1) + 1e-5)
+    assert np.all(np.abs(sl_all[pick] - sl_ref) <= bound[:, sb: sb + span] + 1e-6)
