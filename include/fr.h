@@ -9,8 +9,8 @@
  * sid_base + C_0 + ... + C_{l-1} + c.  A request decodes `depth` steps at beam
  * width K.  At step t every live beam's next-token logits row is normalised
  * with log-softmax over the whole vocabulary V, only the children that the
- * catalog trie allows under the beam's prefix become candidates (illegal SIDs
- * are never candidates), each candidate's score is the beam's running score
+ * catalog trie allows under the beam's prefix become candidates (no token
+ * sequence outside the catalog can be proposed), each candidate's score is the beam's running score
  * plus the child token's log-probability, and the K best candidates of the
  * request survive under a strict total order: higher score first, then lower
  * parent slot, then lower token.  Each survivor records its parent slot (for
@@ -74,8 +74,8 @@ typedef struct fr_beam fr_beam; /* opaque, library-owned */
 const char* fr_status_string(fr_status s);
 
 /* ------------------------------------------------------------------------ */
-/* Catalog trie.  "flashrec 0.1.1 METADATA" §Features/Decoding: the catalog of
- * valid SIDs is held as a CSR-sparse trie and restricts every continuation.
+/* Catalog trie.  "flashrec 0.1.1 METADATA" §Features/Decoding: decoding is
+ * confined to the catalog's valid SIDs through a trie, kept here in CSR form.
  *
  * Layout built on the device: level l (0..depth) holds the distinct length-l
  * SID prefixes in lexicographic order (level 0 = the root alone, level depth
@@ -107,8 +107,8 @@ fr_status fr_trie_level_sizes(const fr_trie* trie, int64_t* nodes_per_level);
 fr_status fr_trie_info(const fr_trie* trie, int32_t* depth, int32_t* sid_base,
                        int32_t* codebook_sizes, int32_t* max_fanout);
 
-/* Dense levels ("flashrec 0.1.1 METADATA", §Architecture: the fused kernel
- * walks a dense or a CSR-sparse trie).  Level l is dense when every level-l
+/* Dense levels ("flashrec 0.1.1 METADATA", §Features/Decoding: the constraint
+ * kernel may work on a dense trie as well as on a sparse CSR one).  Level l is dense when every level-l
  * node has all C_l children (nodes[l+1] == nodes[l] * C_l), detected at build
  * time; the step kernels then index it directly (child of node n with code c
  * = n * C_l + c) instead of reading child_off / code.  The CSR arrays are
@@ -241,17 +241,17 @@ fr_status fr_beam_set_state(fr_beam* beam, int32_t steps_done, const int32_t* li
                             const int32_t* kv_host, fr_stream stream);
 
 /* Normalisation set of the following steps (default FR_NORM_FULL).
- * "flashrec 0.1.1 METADATA", §Features/Decoding: lm_head is evaluated only
- * over the SID token range (FR_NORM_SID_RANGE: each live row streams only
- * that range); "Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation step 4:
- * probabilities over the candidate slice (FR_NORM_CANDIDATES: a beam's
+ * "flashrec 0.1.1 METADATA", §Features/Decoding: the projection is confined
+ * to the ids of the SID tokens (FR_NORM_SID_RANGE: each live row streams only
+ * that range); "Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation step 4: the
+ * softmax is normalised across the candidates alone (FR_NORM_CANDIDATES: a beam's
  * log-softmax runs over its allowed children, at temperature 1; no row is
  * streamed).  Host-side setting; takes effect at the next fr_beam_step. */
 fr_status fr_beam_set_normalization(fr_beam* beam, fr_norm norm);
 
 /* Sampling of the following steps ("flashrec 0.1.1 METADATA", §Serving/API:
- * deterministic top-k at temperature 0, Gumbel top-k without replacement
- * above it).  temperature == 0 (the default) keeps the deterministic top-K.
+ * exact ranking when the temperature is zero; for a positive temperature, K
+ * draws without replacement by Gumbel perturbation of the scores).  temperature == 0 (the default) keeps the deterministic top-K.
  * temperature > 0 ranks each candidate by key = score / temperature + G,
  * where G = -log(-log U) and U = ((u >> 40) + 1/2) * 2^-24, with
  *   u = splitmix64(splitmix64(splitmix64(splitmix64(seed) ^ b') ^ t) ^ (k * 2^32 + token)),

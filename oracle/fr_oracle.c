@@ -14,8 +14,9 @@
  * Sources (page title, section):
  *  - "flashrec 0.1.1 METADATA", opening section and §Features/Decoding: an
  *    item is a short fixed-depth SID token sequence; each continuation is
- *    restricted to the valid-SID catalog ("SID constraint"), so illegal SIDs
- *    are never candidates; wide beam; deterministic top-k at temperature 0.
+ *    restricted to the valid-SID catalog ("SID constraint"), so no SID
+ *    outside the catalog is ever proposed; a wide beam; exact top-K ranking
+ *    when the temperature is zero.
  *  - "beamgrad 2.0.0 PKG-INFO", first code example and §Features: each step
  *    scores the beams' next tokens with log_softmax over the vocabulary
  *    ([B, K, V]); every live beam proposes its continuations, the running
@@ -29,8 +30,9 @@
  *    other K-1 slots dead;
  *  - total order: key descending, then parent slot ascending, then token
  *    ascending; the key is the running score at temperature 0;
- *  - temperature T > 0 ("flashrec 0.1.1 METADATA", §Serving/API: Gumbel
- *    top-k without replacement above temperature 0): each step ranks a
+ *  - temperature T > 0 ("flashrec 0.1.1 METADATA", §Serving/API: a positive
+ *    temperature samples K beams without replacement through Gumbel
+ *    perturbation): each step ranks a
  *    candidate by key = score / T + G with G an independent Gumbel(0, 1)
  *    draw per (request, step, parent slot, token) from a counter-based
  *    SplitMix64 stream (orc_gumbel); survivors keep their unperturbed score
@@ -60,11 +62,11 @@
 /* Normalisation sets of the step's log-softmax:
  *  FULL       the whole vocabulary (the default reading);
  *  SID_RANGE  the SID token range [sid_base, sid_base + C_0 + ... + C_{D-1})
- *             ("flashrec 0.1.1 METADATA", §Features/Decoding: lm_head is
- *             evaluated only over the SID token range);
+ *             ("flashrec 0.1.1 METADATA", §Features/Decoding: the
+ *             projection covers only the ids of the SID tokens);
  *  CANDIDATES the beam's allowed children ("Qwen-2.5-1B-RLCD-Fast",
- *             §Parallel Evaluation step 4: probabilities over the candidate
- *             slice), at temperature 1. */
+ *             §Parallel Evaluation step 4: the softmax is normalised across
+ *             the candidates alone), at temperature 1. */
 #define ORC_NORM_FULL 0
 #define ORC_NORM_SID_RANGE 1
 #define ORC_NORM_CANDIDATES 2

@@ -1,5 +1,5 @@
-"""Dense trie levels ("flashrec 0.1.1 METADATA", §Architecture: the fused
-kernel walks a dense or a CSR-sparse trie).  Where every node of a level has
+"""Dense trie levels ("flashrec 0.1.1 METADATA", §Features/Decoding: the
+constraint kernel may work on a dense trie as well as on a sparse one).  Where every node of a level has
 all C_l children the step kernels index the level directly instead of reading
 its CSR arrays.  Detection is checked against the catalog's own child counts;
 the lookups are integer work, so a decode with direct indexing must be

@@ -1,6 +1,6 @@
 """The two other normalisation sets the pages describe, on the GPU vs the
 oracle: the SID token range ("flashrec 0.1.1 METADATA", §Features/Decoding:
-lm_head is evaluated only over the SID token range) and the candidate slice
+the projection covers only the ids of the SID tokens) and the candidate slice
 ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation step 4).  Same near-tie
 protocol and tolerance as the full-vocabulary tests."""
 import numpy as np

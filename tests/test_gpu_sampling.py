@@ -1,6 +1,6 @@
 """Sampling above temperature 0 on the GPU vs the oracle ("flashrec 0.1.1
-METADATA", §Serving/API: deterministic top-k at temperature 0, Gumbel top-k
-without replacement above it).
+METADATA", §Serving/API: exact ranking at temperature zero, sampling without
+replacement by Gumbel perturbation at a positive temperature).
 
 Both sides draw the same Gumbel noise (one counter-based SplitMix64 stream,
 indexed by request, step, parent slot and token), so the sampled beams are

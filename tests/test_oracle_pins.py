@@ -6,7 +6,8 @@ torch's conversion, a library routine), exactness of the hash logits, brute
 force enumeration when nothing can be pruned (K >= catalog size), greedy
 constrained decoding (K = 1), the all-equal-logits closed form, and the
 invariants the pages state (every emitted SID is in the catalog --
-"flashrec 0.1.1 METADATA", §Features: illegal SIDs are never candidates).
+"flashrec 0.1.1 METADATA", §Features: no SID outside the catalog is ever
+proposed).
 """
 import math
 import os

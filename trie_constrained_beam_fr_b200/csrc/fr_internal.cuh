@@ -22,8 +22,8 @@ struct TrieDev {
     const int32_t* leaf_row;                    // [nodes[depth]]
     int32_t nodes[FR_MAX_DEPTH + 1];
     int32_t tok_base[FR_MAX_DEPTH];             // token id of (level l, code 0)
-    // Dense levels ("flashrec 0.1.1 METADATA", §Architecture: dense or
-    // CSR-sparse trie): C_l when every level-l node has all C_l children (so
+    // Dense levels ("flashrec 0.1.1 METADATA", §Features/Decoding: a dense
+    // trie as well as a sparse one): C_l when every level-l node has all C_l children (so
     // child_off[l][n] = n * C_l and the child's code is its index mod C_l),
     // else 0 (look the level up in the CSR arrays).
     int32_t dense_c[FR_MAX_DEPTH];

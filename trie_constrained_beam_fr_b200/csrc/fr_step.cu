@@ -32,8 +32,8 @@
 //            reorder gathers: backpointer, token, trie node, score, prefix and
 //            KV slot of every survivor, and the next step's candidate offsets.
 //
-// Above temperature 0 ("flashrec 0.1.1 METADATA", §Serving/API: Gumbel top-k
-// without replacement) the candidate writers also store a perturbed key
+// Above temperature 0 ("flashrec 0.1.1 METADATA", §Serving/API: sampling
+// without replacement by Gumbel perturbation) the candidate writers also store a perturbed key
 // score / T + G per candidate, G a Gumbel(0, 1) draw from a counter-based
 // SplitMix64 stream indexed by (request, step, parent slot, token); k_select
 // ranks the keys and the survivors keep their unperturbed scores.
@@ -868,7 +868,7 @@ __global__ void __launch_bounds__(256) k_rows_given_lse(const StreamArgs a) {
 
 // ---------------------------------------------------------------------------
 // Candidate-slice normalisation ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation
-// step 4: probabilities over the candidate slice): a beam's log-softmax runs
+// step 4: the softmax normalised across the candidates alone): a beam's log-softmax runs
 // over its allowed children only, so no logits row is streamed.  One warp per
 // live beam gathers the children's logits, takes their log-sum-exp and writes
 // the candidate scores s_k + (x - lse_slice).

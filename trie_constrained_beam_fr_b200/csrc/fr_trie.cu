@@ -1,7 +1,7 @@
 // fr_trie.cu -- device construction of the CSR catalog trie.
 //
-// "flashrec 0.1.1 METADATA", §Features/Decoding: decoding is restricted to a
-// catalog of valid SIDs held as a dense or CSR-sparse trie.  This builds the
+// "flashrec 0.1.1 METADATA", §Features/Decoding: decoding is confined to the
+// catalog's valid SIDs through a trie (dense, or sparse in CSR form).  This builds the
 // CSR form on the GPU:
 //   1. pack each SID into one 64-bit key, level 0 in the highest bits, and
 //      check every code against its codebook size;
