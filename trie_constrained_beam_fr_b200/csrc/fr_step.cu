@@ -1477,11 +1477,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
 // ---------------------------------------------------------------------------
 // State kernels.
 
-__global__ void k_reset(StateDev s0, int32_t B, int32_t K, int32_t D, TrieDev trie) {
+__global__ void k_reset(StateDev s0, StepBuffers buf, int32_t B, int32_t K, int32_t D, TrieDev trie) {
     const int64_t nbk = (int64_t)B * K;
     int32_t root_lo, root_hi;
     trie_children(trie, 0, 0, root_lo, root_hi);
     const int32_t root_fan = root_hi - root_lo;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *buf.err = 0;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
         const int32_t b = (int32_t)(i / K), k = (int32_t)(i % K);
         const bool root = (k == 0);
@@ -1490,6 +1491,9 @@ __global__ void k_reset(StateDev s0, int32_t B, int32_t K, int32_t D, TrieDev tr
         s0.kv[i] = root ? b * K : -1;
         for (int l = 0; l < D; ++l) s0.prefix[i * D + l] = -1;
         if (root) s0.live[b] = 1;
+        buf.parent[i] = -1;
+        buf.token[i] = -1;
+        buf.row_cnt[i] = 0;
     }
     const int64_t no = (int64_t)B * (K + 1);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < no; i += (int64_t)gridDim.x * blockDim.x) {
@@ -1796,13 +1800,8 @@ int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {
 
 cudaError_t launch_reset(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, cudaStream_t s) {
     const int64_t nbk = (int64_t)sh.B * sh.K;
-    k_reset<<<small_grid(nbk + sh.B), 256, 0, s>>>(buf.st[0], sh.B, sh.K, sh.D, trie);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(buf.parent, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(buf.token, 0xFF, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(buf.row_cnt, 0, sizeof(int32_t) * (size_t)nbk, s)) != cudaSuccess) return e;
-    return cudaMemsetAsync(buf.err, 0, sizeof(int32_t), s);
+    k_reset<<<small_grid(nbk + sh.B), 256, 0, s>>>(buf.st[0], buf, sh.B, sh.K, sh.D, trie);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_set_state(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
