@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 W = synth.Workload
 # Rows whose streamed window is at most 16 KB take the warp-per-row kernel
 # (tiny, ragged_bf16, k1024, greedy, k_exceeds_catalog, k1024_wide_fanout,
-# cluster2, cluster4, deep); longer rows take the persistent streaming kernel
+# cluster2, cluster4, deep, odd_stride, narrow_ties); longer rows take the persistent streaming kernel
 # (ragged_wide_bf16, mid_bf16, mid_f32_deep, full_vocab_few_rows,
 # skewed_small, max_requests).  Selections over more than 16,384 candidates
 # per request run in thread-block clusters: k1024 and skewed_small (8 CTAs),
@@ -61,6 +61,15 @@ SMALL = {
     # a deep trie: 12 levels of 4 codes
     "deep": W("deep", B=2, K=16, depth=12, C=4, V=200, sid_base=100, n_items=5000, dtype="bf16", seed=14,
               catalog_seed=14),
+    # K x max fan-out = 3 x 9 candidates per request: the candidate rows' stride
+    # is rounded up to 28 so that each request's row starts on 16 bytes
+    "odd_stride": W("odd_stride", B=3, K=3, depth=2, C=16, V=64, sid_base=16, n_items=11, dtype="f32", seed=23,
+                    catalog_seed=23),
+    # 80 requests (too many for clusters) of ~19,500 candidates at step 1, in
+    # one CTA each from L2; bf16 logits repeat among a parent's ~390 children,
+    # so equal scores often straddle the K-th place
+    "narrow_ties": W("narrow_ties", B=80, K=50, depth=2, C=1024, V=2100, sid_base=30, n_items=400_000,
+                     dtype="bf16", seed=16, catalog_seed=16),
     # K x max fan-out = 1024 x 1024 candidates: beyond what a 16-CTA cluster
     # holds in shared memory, so the selection reads the candidates from L2
     "k1024_wide_fanout": W("k1024_wide_fanout", B=2, K=1024, depth=2, C=1024, V=2100, sid_base=30,

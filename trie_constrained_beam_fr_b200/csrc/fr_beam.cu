@@ -100,7 +100,9 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
         bm->shape.sel_cluster[t] = fr::select_cluster_size(B, K, bound, sms);
     }
     const size_t bk = (size_t)B * K;
-    const int64_t cand_stride = (int64_t)K * std::max(1, trie->max_fanout);
+    // a request's candidates: K beams x the widest fan-out, rounded up to a
+    // multiple of 4 so that every request's row starts on 16 bytes
+    const int64_t cand_stride = ((int64_t)K * std::max(1, trie->max_fanout) + 3) & ~(int64_t)3;
     size_t bytes = 0;
     for (int i = 0; i < 2; ++i) {
         bytes += align256(sizeof(int32_t) * bk);      // node

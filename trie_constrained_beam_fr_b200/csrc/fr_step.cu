@@ -1130,38 +1130,99 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
 // order-preserving image of the candidate's score (or sampling key) and low =
 // ~slot, so that larger values come first in the step's total order (key
 // descending, slot ascending) and index order is slot order.
-struct GlobalCands {  // the request's candidates in global memory, slot i at cb[i]
+// QUADS: keys 4q .. 4q+3 come from one 16-byte load, key4(q).  val_of(i, k)
+// is val(i) for a key k already loaded.
+struct GlobalCands {  // the request's candidates in global memory, slot i at cb[i] (cb 16-byte aligned)
+    static constexpr bool QUADS = true;
     const float* cb;
     __device__ __forceinline__ uint32_t key(int i) const { return float_to_key(__ldg(cb + i)); }
-    __device__ __forceinline__ unsigned long long val(int i) const {
-        return ((unsigned long long)key(i) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+    __device__ __forceinline__ uint4 key4(int q) const {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(cb) + q);
+        return make_uint4(float_to_key(x.x), float_to_key(x.y), float_to_key(x.z), float_to_key(x.w));
     }
+    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t k) const {
+        return ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
+    }
+    __device__ __forceinline__ unsigned long long val(int i) const { return val_of(i, key(i)); }
 };
 struct SmemKeys {  // a contiguous slice of them, as keys in shared memory, slot base + i at keys[i]
+    static constexpr bool QUADS = false;
     const uint32_t* keys;
     uint32_t base;
     __device__ __forceinline__ uint32_t key(int i) const { return keys[i]; }
-    __device__ __forceinline__ unsigned long long val(int i) const {
-        return ((unsigned long long)keys[i] << 32) | (0xFFFFFFFFu - (base + (uint32_t)i));
+    __device__ __forceinline__ uint4 key4(int) const { return make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t k) const {
+        return ((unsigned long long)k << 32) | (0xFFFFFFFFu - (base + (uint32_t)i));
     }
+    __device__ __forceinline__ unsigned long long val(int i) const { return val_of(i, keys[i]); }
 };
 struct PoolVals {  // values already formed, in slot order
+    static constexpr bool QUADS = false;
     const unsigned long long* pool;
     __device__ __forceinline__ uint32_t key(int i) const { return (uint32_t)(pool[i] >> 32); }
+    __device__ __forceinline__ uint4 key4(int) const { return make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t) const { return pool[i]; }
     __device__ __forceinline__ unsigned long long val(int i) const { return pool[i]; }
 };
+
+// Calls f(i, key(i)) for the indices i in [0, n) this thread owns (which ones
+// depends on the access width), with eight independent loads in flight per
+// thread.  The calls' order is not index order.
+template <class Vals, class F>
+__device__ __forceinline__ void for_keys(const Vals& vals, int n, F&& f) {
+    const int tid = threadIdx.x;
+    if constexpr (Vals::QUADS) {
+        const int nq = n >> 2;
+        int q0 = tid;
+        for (; q0 + 7 * SEL_THREADS < nq; q0 += 8 * SEL_THREADS) {
+            uint4 k4[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) k4[u] = vals.key4(q0 + u * SEL_THREADS);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = (q0 + u * SEL_THREADS) * 4;
+                f(i, k4[u].x);
+                f(i + 1, k4[u].y);
+                f(i + 2, k4[u].z);
+                f(i + 3, k4[u].w);
+            }
+        }
+        for (int q = q0; q < nq; q += SEL_THREADS) {
+            const uint4 k4 = vals.key4(q);
+            f(4 * q, k4.x);
+            f(4 * q + 1, k4.y);
+            f(4 * q + 2, k4.z);
+            f(4 * q + 3, k4.w);
+        }
+        const int i = 4 * nq + tid;  // the last n mod 4
+        if (i < n) f(i, vals.key(i));
+    } else {
+        int i0 = tid;
+        for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
+            uint32_t k8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) k8[u] = vals.key(i0 + u * SEL_THREADS);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f(i0 + u * SEL_THREADS, k8[u]);
+        }
+        for (int i = i0; i < n; i += SEL_THREADS) f(i, vals.key(i));
+    }
+}
 
 // Exact top-Kp (Kp <= n, Kp <= FR_MAX_K) of the n values under the total
 // order: the Kp winners' values go to out[0..Kp); the return value is how
 // many were written (Kp unless something is inconsistent).  The Kp-th key T
 // is found by radix selection on the keys (12-bit digits after skipping the
 // bits every key shares); the winners are every key > T and the lowest-index
-// keys == T.  ORDERED: they are written in index (slot) order -- each warp
+// keys == T.  The search stops early once the bin holding the Kp-th key holds
+// exactly the keys still needed: T is then that bin's lowest value, and the
+// winners are the keys >= T.  ORDERED: they are written in index (slot) order -- each warp
 // owns a contiguous block of indices and counts its keys above and at T
 // (ballots), one scan over the warps gives each warp its output offset, and a
 // second sweep writes.  Otherwise in any order, in one sweep (atomic
-// positions; the keys equal to T are taken in index order, by block scans,
-// only when not all of them win).  All threads of the block call it; scratch:
+// positions; when not all the keys equal to T win, their lowest indices are
+// found by ranking them, or, past SEL_THREADS of them, by block scans in index
+// order).  All threads of the block call it; scratch:
 // hist [HBINS], red [64], s_misc [8].
 template <bool ORDERED, class Vals>
 __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* out, int32_t* hist, uint32_t* red,
@@ -1173,22 +1234,10 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
     int count_eq = n;   // keys equal to T (an upper bound when every value wins)
     if (Kp < n) {
         uint32_t va = 0xFFFFFFFFu, vo = 0u;
-        int i0 = tid;
-        for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-            uint32_t k8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) k8[u] = vals.key(i0 + u * SEL_THREADS);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                va &= k8[u];
-                vo |= k8[u];
-            }
-        }
-        for (int i = i0; i < n; i += SEL_THREADS) {
-            const uint32_t k = vals.key(i);
+        for_keys(vals, n, [&](int, uint32_t k) {
             va &= k;
             vo |= k;
-        }
+        });
         uint32_t VO;
         const uint32_t VA = block_and_or(va, vo, red, &VO);
         const uint32_t diff = VA ^ VO;
@@ -1207,19 +1256,9 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
                 for (int i = tid; i < HBINS; i += SEL_THREADS) hist[i] = 0;
                 __syncthreads();
                 const uint64_t want = (uint64_t)prefix >> lo;
-                int j0 = tid;
-                for (; j0 + 7 * SEL_THREADS < n; j0 += 8 * SEL_THREADS) {
-                    uint32_t k8[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) k8[u] = vals.key(j0 + u * SEL_THREADS);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (((uint64_t)k8[u] >> lo) == want) atomicAdd(&hist[(k8[u] >> shift) & dmask], 1);
-                }
-                for (int i = j0; i < n; i += SEL_THREADS) {
-                    const uint32_t k = vals.key(i);
+                for_keys(vals, n, [&](int, uint32_t k) {
                     if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
-                }
+                });
                 __syncthreads();
                 int h4[4], tsum = 0;
 #pragma unroll
@@ -1245,35 +1284,53 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
                 prefix |= (uint32_t)s_misc[0] << shift;
                 lo = shift;
                 __syncthreads();
+                // Every key of the threshold bin wins: T = prefix (its lower
+                // bits zero) already splits the keys, with keys >= T winning.
+                if (count_eq == krem) break;
             }
             T = prefix;
             eq_needed = krem;
         }
     }
     if constexpr (!ORDERED) {
-        if (tid == 0) s_misc[3] = 0;
+        if (tid == 0) {
+            s_misc[3] = 0;
+            s_misc[4] = 0;
+        }
         __syncthreads();
         if (eq_needed >= count_eq) {  // every key >= T wins
-            int i0 = tid;
-            for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-                unsigned long long v8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v8[u] = vals.val(i0 + u * SEL_THREADS);
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if ((uint32_t)(v8[u] >> 32) >= T) {
-                        const int p = atomicAdd(&s_misc[3], 1);
-                        if (p < Kp) out[p] = v8[u];
-                    }
-            }
-            for (int i = i0; i < n; i += SEL_THREADS) {
-                const unsigned long long v = vals.val(i);
-                if ((uint32_t)(v >> 32) >= T) {
+            for_keys(vals, n, [&](int i, uint32_t k) {
+                if (k >= T) {
                     const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < Kp) out[p] = v;
+                    if (p < Kp) out[p] = vals.val_of(i, k);
+                }
+            });
+        } else if (count_eq <= SEL_THREADS) {
+            // Few keys equal T (ties of equal scores): every key > T wins;
+            // the indices of the keys == T go to the histogram's space, and
+            // those with fewer than eq_needed lower indices among them win.
+            int32_t* eq_idx = hist;
+            for_keys(vals, n, [&](int i, uint32_t k) {
+                if (k > T) {
+                    const int p = atomicAdd(&s_misc[3], 1);
+                    if (p < Kp) out[p] = vals.val_of(i, k);
+                } else if (k == T) {
+                    const int q = atomicAdd(&s_misc[4], 1);
+                    if (q < SEL_THREADS) eq_idx[q] = i;
+                }
+            });
+            __syncthreads();
+            const int ne = min(s_misc[4], SEL_THREADS);
+            if (tid < ne) {
+                const int mine = eq_idx[tid];
+                int below = 0;
+                for (int j = 0; j < ne; ++j) below += eq_idx[j] < mine;
+                if (below < eq_needed) {
+                    const int p = atomicAdd(&s_misc[3], 1);
+                    if (p < Kp) out[p] = vals.val_of(mine, T);
                 }
             }
-        } else {  // the keys equal to T straddle the boundary: take them in index order
+        } else {  // many keys equal T straddle the boundary: take them in index order
             int run_eq = 0;
             for (int base = 0; base < n; base += SEL_THREADS) {
                 const int i = base + tid;

@@ -14,7 +14,7 @@ struct StepBuffers {
     int32_t* token;       // [B*K]
     float* cand;          // [B * cand_stride] candidate scores
     float* cand_key;      // [B * cand_stride] perturbed keys (sampling above temperature 0)
-    int64_t cand_stride;  // K * max_fanout
+    int64_t cand_stride;  // K * max_fanout rounded up to a multiple of 4
     float2* partial;      // [grid * 2] (max, scaled sum) per CTA and row side
     int32_t* row_cnt;     // [B*K] arrival counters of shared rows
     int32_t* err;         // sticky device status word
