@@ -31,7 +31,9 @@ from trie_constrained_beam_fr_b200 import synth  # noqa: E402
 
 METRIC = "constrained beam candidates/sec (B·K·steps/s) and logits HBM GB/s vs 8 TB/s"
 UNIT = "candidates/s"
-STREAM_KERNEL_SRC = os.path.join(ROOT, "trie_constrained_beam_fr_b200", "csrc", "fr_step.cu")
+# the streaming kernel's translation unit: its source and the headers it includes
+STREAM_KERNEL_SRC = [os.path.join(ROOT, "trie_constrained_beam_fr_b200", "csrc", f)
+                     for f in ("fr_step.cu", "fr_step.cuh", "fr_internal.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -96,13 +98,16 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the streaming kernel's source with comments and blank lines
-    removed: recorded counters stay valid across comment-only edits and are
-    dropped as soon as any code changes."""
+    """Hash of the streaming kernel's sources (its file and the headers it
+    includes) with comments and blank lines removed: recorded counters stay
+    valid across comment-only edits and are dropped as soon as any code
+    changes."""
     import re
 
-    with open(STREAM_KERNEL_SRC) as f:
-        src = f.read()
+    src = ""
+    for path in STREAM_KERNEL_SRC:
+        with open(path) as f:
+            src += f.read() + "\n"
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
     code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())

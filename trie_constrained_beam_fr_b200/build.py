@@ -25,7 +25,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 
 TARGETS = {
-    "libfr.so": ["fr_trie.cu", "fr_step.cu", "fr_beam.cu", "fr_noalloc.cu", "fr_lmhead.cu"],
+    "libfr.so": ["fr_trie.cu", "fr_step.cu", "fr_select.cu", "fr_beam.cu", "fr_noalloc.cu", "fr_lmhead.cu"],
     "libfr_gen.so": ["fr_gen.cu"],
 }
 HEADERS = ["fr_internal.cuh", "fr_handles.h", "fr_step.cuh"]

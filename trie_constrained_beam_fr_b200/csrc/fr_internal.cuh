@@ -136,6 +136,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Programmatic dependent launch (sm_90 and later).  The step kernels are
+// launched with programmatic stream serialization, so a kernel may be
+// scheduled while the previous kernel of the stream is still running: it first
+// waits (griddep_wait) until that kernel has completed and its memory is
+// visible, then allows the next kernel to be scheduled
+// (griddep_launch_dependents).  The next kernel is released only once every
+// CTA of this one has signalled, so it never takes resources this grid still
+// needs.  For a kernel launched without the attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ int warp_incl_scan(int v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll

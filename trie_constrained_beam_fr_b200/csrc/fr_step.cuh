@@ -33,6 +33,40 @@ struct StepShape {
     int64_t req_offset;  // index of local request 0 in the Gumbel stream
 };
 
+// Launch configuration of a step kernel: programmatic stream serialization
+// (see griddep_wait), and optionally a cluster size.  Used in place (cfg
+// points into the object).
+struct StepLaunch {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[2];
+    StepLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster = 0) {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        int n = 1;
+        if (cluster) {
+            attr[1].id = cudaLaunchAttributeClusterDimension;
+            attr[1].val.clusterDim.x = cluster;
+            attr[1].val.clusterDim.y = 1;
+            attr[1].val.clusterDim.z = 1;
+            n = 2;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = n;
+    }
+    StepLaunch(const StepLaunch&) = delete;
+    StepLaunch& operator=(const StepLaunch&) = delete;
+};
+
+// Blocks of 256 threads covering n items (grid-stride beyond 4096 blocks).
+inline int small_grid(int64_t n) {
+    const int64_t g = (n + 255) / 256;
+    return (int)(g < 1 ? 1 : (g > 4096 ? 4096 : g));
+}
+
 // Cluster size of the selection for a step whose requests have at most
 // `bound` candidates (0 = the single-CTA kernel).
 int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms);
