@@ -207,6 +207,49 @@ class ClockSampler:
 NORM_CODES = {"full": 0, "sid_range": 1, "candidates": 2}  # fr_norm values (include/fr.h)
 
 
+def catalog_level_sizes(sids: np.ndarray) -> list:
+    """Nodes per trie level of a catalog: the root, then the distinct SID
+    prefixes of each length (the level sizes the device trie build reports)."""
+    u = np.unique(sids, axis=0)
+    return [1] + [int(np.unique(u[:, : l + 1], axis=0).shape[0]) for l in range(u.shape[1])]
+
+
+def logits_config(w: synth.Workload, args, levels) -> dict:
+    """`config` of a bench line on the logits path (both arms)."""
+    return {"workload": w.name, "norm": args.norm, "temperature": args.temperature, "B_per_gpu": w.B, "K": w.K,
+            "depth": w.depth, "V": w.V, "codes_per_level": w.C, "catalog": w.n_items, "logits": w.dtype,
+            "trie_levels": list(levels),
+            "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"
+                  % (w.B * w.K * w.V * w.elt_size / 1e9),
+            "step": "one full decode: depth beam steps + finalize"}
+
+
+def lmhead_config(w: synth.Workload, args) -> dict:
+    """`config` of a bench line on the lm_head path (both arms)."""
+    dh = args.lmhead
+    return {"workload": w.name, "path": "lm_head", "hidden_size": dh, "norm": args.norm,
+            "temperature": args.temperature, "B_per_gpu": w.B, "K": w.K, "depth": w.depth, "V": w.V,
+            "codes_per_level": w.C, "catalog": w.n_items,
+            "l2": "per step a distinct %.0f MB hidden-state buffer; the %.0f MB lm_head is re-read "
+                  "every step (larger than L2)" % (w.B * w.K * dh * 2 / 1e6, w.V * dh * 2 / 1e6),
+            "step": "one full decode: depth x (fused lm_head + beam step) + finalize"}
+
+
+def lmhead_oracle_sample(w: synth.Workload, hidden: np.ndarray, weight: np.ndarray) -> dict:
+    """The oracle's lm_head rows for the given rows of one request, timed, and
+    scaled to that request's decode: 1 row at step 0, K at every later step.
+    The selection's cost is negligible next to the rows."""
+    import oracle
+
+    span = sum(w.codebook_sizes)
+    t0 = time.perf_counter()
+    oracle.lmhead_rows(hidden, weight, w.sid_base, span)
+    per_row = (time.perf_counter() - t0) / hidden.shape[0]
+    rows_per_request = 1 + (w.depth - 1) * w.K
+    return {"candidates": w.K * w.depth, "method_s": rows_per_request * per_row, "per_row_s": per_row,
+            "rows_per_request": rows_per_request}
+
+
 def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, sids=None, cat=None,
                   norm: str = "full", temperature: float = 0.0):
     import oracle
@@ -226,31 +269,51 @@ def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, si
 
 
 def run_reference(args):
+    """The oracle on host cores, on the same workload, config, metric and
+    unit as the GPU arm; each step a bounded sample of that workload."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import oracle
 
     w = synth.WORKLOADS[args.config]
+    if args.batch:
+        w = synth.scaled(w, B=args.batch)
     sids = synth.workload_catalog(w)
-    cat = oracle.Catalog(sids, w.codebook_sizes)
-    for i in range(args.warmup):
-        oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
-                      temperature=args.temperature)
-    samples = [oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
-                             temperature=args.temperature)
-               for i in range(args.steps)]
+    if args.lmhead:
+        dh = args.lmhead
+        rng = np.random.default_rng(1234)
+        # bf16-representable values of the GPU arm's scale; only the timing is used
+        weight = (rng.integers(-128, 128, size=(w.V, dh), dtype=np.int16).astype(np.float32) / 8192.0)
+        n_rows = 4
+        hid = [rng.integers(-128, 128, size=(n_rows, dh), dtype=np.int16).astype(np.float32) / 64.0
+               for _ in range(args.warmup + args.steps)]
+        for i in range(args.warmup):
+            lmhead_oracle_sample(w, hid[i], weight)
+        samples = [lmhead_oracle_sample(w, hid[args.warmup + i], weight) for i in range(args.steps)]
+        config = lmhead_config(w, args)
+        sample = ("oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of one request "
+                  "per step, scaled to that request's decode (%d rows)"
+                  % (w.V, dh, n_rows, samples[0]["rows_per_request"]))
+    else:
+        cat = oracle.Catalog(sids, w.codebook_sizes)
+        for i in range(args.warmup):
+            oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
+                          temperature=args.temperature)
+        samples = [oracle_sample(w, args.ref_requests, first_request=i % w.B, sids=sids, cat=cat, norm=args.norm,
+                                 temperature=args.temperature)
+                   for i in range(args.steps)]
+        config = logits_config(w, args, catalog_level_sizes(sids))
+        sample = ("%d request(s) of %s per step (of B=%d), full decode, oracle time excluding its logits generation"
+                  % (args.ref_requests, w.name, w.B))
     cand = sum(s["candidates"] for s in samples)
     secs = sum(s["method_s"] for s in samples)
     value = cand / secs
-    sample = ("%d request(s) of %s per step (of B=%d), full decode, oracle time excluding its logits generation"
-              % (args.ref_requests, w.name, w.B))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "norm": args.norm, "temperature": args.temperature, "B": w.B, "K": w.K, "depth": w.depth, "V": w.V, "codes_per_level": w.C,
-                   "catalog": w.n_items, "logits": w.dtype},
+        "config": config,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -394,32 +457,20 @@ def run_lmhead(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-
         n = 4
-        hh = hidden[1][0, :n].float().cpu().numpy()
-        ww = weight.float().cpu().numpy()
-        c0 = time.perf_counter()
-        oracle.lmhead_rows(hh, ww, w.sid_base, span)
-        per_row = (time.perf_counter() - c0) / n
-        rows_per_request = 1 + (D - 1) * K
-        cpu = {"value": K * D / (rows_per_request * per_row), "unit": UNIT, "cores": 1, "kind": "oracle",
+        s = lmhead_oracle_sample(w, hidden[1][0, :n].float().cpu().numpy(), weight.float().cpu().numpy())
+        cpu = {"value": s["candidates"] / s["method_s"], "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of "
                          "request 0, %.2f s per row, scaled to one request's decode (%d rows: 1 at step 0, "
                          "K afterwards); the selection's cost is negligible next to the rows"
-                         % (V, dh, n, per_row, rows_per_request)}
+                         % (V, dh, n, s["per_row_s"], s["rows_per_request"])}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
-            "config": {"workload": w.name, "path": "lm_head", "hidden_size": dh, "norm": args.norm,
-                       "temperature": args.temperature, "B_per_gpu": B, "K": K, "depth": D, "V": V,
-                       "codes_per_level": w.C, "catalog": w.n_items,
-                       "l2": "per step a distinct %.0f MB hidden-state buffer; the %.0f MB lm_head is re-read "
-                             "every step (larger than L2)" % (B * K * dh * 2 / 1e6, V * dh * 2 / 1e6),
-                       "step": "one full decode: depth x (fused lm_head + beam step) + finalize"},
+            "config": lmhead_config(w, args),
             "roofline": roofline, "per_step": per_step, "gpu_launches": args.steps * (4 * D + 2),
             "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu,
         }
@@ -637,12 +688,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "norm": args.norm, "temperature": args.temperature, "B_per_gpu": B, "K": K, "depth": D, "V": V,
-                       "codes_per_level": w.C,
-                       "catalog": w.n_items, "logits": w.dtype, "trie_levels": levels,
-                       "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"
-                             % (B * K * V * elt / 1e9),
-                       "step": "one full decode: depth beam steps + finalize"},
+            "config": logits_config(w, args, levels),
             "hbm_gbs": hbm_gbs_decode, "hbm_frac_of_8tbs": hbm_gbs_decode / 8000.0,
             "ms_per_step_with_kernel_events": evented_ms / args.steps,
             "roofline": roofline, "per_step": per_step, "trie_build_ms": trie_ms,

@@ -1,0 +1,63 @@
+"""The benchmark's reference arm on CPU: the oracle, timed on host cores on a
+bounded sample of the GPU arm's workload.  Its JSON line carries the GPU arm's
+metric, unit, direction and config (one builder serves both arms), a
+cpu_baseline describing the run and an e2e with no host-device traffic; under
+more than one rank only rank 0 runs it."""
+import argparse
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+import bench
+from trie_constrained_beam_fr_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
+                          env=env, timeout=600, cwd=ROOT)
+
+
+def test_reference_line_matches_the_gpu_arm_contract():
+    r = _run(["--impl", "reference", "--config", "serving", "--steps", "1", "--warmup", "0"])
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
+    assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0 and d["data"] == "synthetic"
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+    w = synth.WORKLOADS["serving"]
+    sids = synth.workload_catalog(w)
+    levels = bench.catalog_level_sizes(sids)
+    args = argparse.Namespace(norm="full", temperature=0.0)
+    assert d["config"] == bench.logits_config(w, args, levels)
+    # the level sizes the device build reports: root, then distinct prefixes
+    C = w.codebook_sizes
+    assert levels[0] == 1 and levels[-1] == np.unique(sids, axis=0).shape[0]
+    for l in range(1, len(levels)):
+        assert levels[l - 1] <= levels[l] <= levels[l - 1] * C[l - 1]
+
+
+def test_level_sizes_of_a_hand_catalog():
+    sids = np.array([[0, 1, 2], [0, 1, 3], [0, 2, 0], [5, 0, 0], [0, 1, 2]], np.int32)  # one duplicate
+    assert bench.catalog_level_sizes(sids) == [1, 2, 3, 4]
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    r = _run(["--impl", "reference", "--config", "serving", "--steps", "1", "--warmup", "0"],
+             {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
