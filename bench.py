@@ -268,6 +268,53 @@ def oracle_sample(w: synth.Workload, n_requests: int, first_request: int = 0, si
     return {"candidates": n_requests * w.K * w.depth, "method_s": method, "gen_s": r.gen_seconds, "wall_s": wall}
 
 
+CPU_SAMPLE_S = 10.0  # CPU work of a cpu_baseline sample (the oracle is slow by design)
+
+
+def cpu_baseline_logits(w: synth.Workload, sids: np.ndarray, norm: str, temperature: float,
+                        min_s: float = CPU_SAMPLE_S) -> dict:
+    """cpu_baseline on the logits path: whole decodes of requests 0, 1, ...
+    by the single-threaded oracle until about min_s seconds of CPU work (at
+    least one request, at most B), timing the method without the oracle's
+    own logits generation."""
+    import oracle
+
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    cand, method, gen, n = 0, 0.0, 0.0, 0
+    t0 = time.perf_counter()
+    while n < w.B and (n == 0 or time.perf_counter() - t0 < min_s):
+        smp = oracle_sample(w, 1, first_request=n, sids=sids, cat=cat, norm=norm, temperature=temperature)
+        cand += smp["candidates"]
+        method += smp["method_s"]
+        gen += smp["gen_s"]
+        n += 1
+    return {"value": cand / method, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "requests 0..%d of %s (%d of B=%d), a full decode each, single-threaded C oracle in double, "
+                      "time excluding its logits generation (%.1f s method, %.1f s generation)"
+                      % (n - 1, w.name, n, w.B, method, gen)}
+
+
+def cpu_baseline_lmhead(w: synth.Workload, rows: np.ndarray, weight: np.ndarray,
+                        min_s: float = CPU_SAMPLE_S) -> dict:
+    """cpu_baseline on the lm_head path: the oracle's lm_head rows (float32
+    rows [r, d] of one request) 4 at a time until about min_s seconds, the
+    mean time per row scaled to one request's decode."""
+    done, secs = 0, 0.0
+    per_req = None
+    while done < rows.shape[0] and (done == 0 or secs < min_s):
+        smp = lmhead_oracle_sample(w, rows[done:done + 4], weight)
+        n = min(4, rows.shape[0] - done)
+        secs += smp["per_row_s"] * n
+        done += n
+        per_req = smp["rows_per_request"]
+    per_row = secs / done
+    return {"value": w.K * w.depth / (per_req * per_row), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of "
+                      "request 0, %.2f s per row, scaled to one request's decode (%d rows: 1 at step 0, "
+                      "K afterwards); the selection's cost is negligible next to the rows"
+                      % (w.V, weight.shape[1], done, per_row, per_req)}
+
+
 def run_reference(args):
     """The oracle on host cores, on the same workload, config, metric and
     unit as the GPU arm; each step a bounded sample of that workload."""
@@ -467,13 +514,7 @@ def run_lmhead(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = 4
-        s = lmhead_oracle_sample(w, hidden[1][0, :n].float().cpu().numpy(), weight.float().cpu().numpy())
-        cpu = {"value": s["candidates"] / s["method_s"], "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of "
-                         "request 0, %.2f s per row, scaled to one request's decode (%d rows: 1 at step 0, "
-                         "K afterwards); the selection's cost is negligible next to the rows"
-                         % (V, dh, n, s["per_row_s"], s["rows_per_request"])}
+        cpu = cpu_baseline_lmhead(w, hidden[1][0].float().cpu().numpy(), weight.float().cpu().numpy())
 
     if rank == 0:
         line = {
@@ -686,11 +727,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s = oracle_sample(w, 1, first_request=0, sids=sids_np, norm=args.norm, temperature=args.temperature)
-        cpu = {"value": s["candidates"] / s["method_s"], "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "request 0 of %s (1 of B=%d), full decode, single-threaded C oracle in double, "
-                         "time excluding its logits generation (%.1f s method, %.1f s generation)"
-                         % (w.name, w.B, s["method_s"], s["gen_s"])}
+        cpu = cpu_baseline_logits(w, sids_np, args.norm, args.temperature)
 
     if rank == 0:
         line = {

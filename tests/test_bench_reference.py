@@ -2,7 +2,8 @@
 bounded sample of the GPU arm's workload.  Its JSON line carries the GPU arm's
 metric, unit, direction and config (one builder serves both arms), a
 cpu_baseline describing the run and an e2e with no host-device traffic; under
-more than one rank only rank 0 runs it."""
+more than one rank only rank 0 runs it.  The GPU arm's cpu_baseline legs
+sample whole requests (or lm_head rows) up to a CPU-time budget."""
 import argparse
 import json
 import os
@@ -61,3 +62,24 @@ def test_reference_arm_runs_on_rank_zero_only():
              {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_cpu_baseline_samples_whole_requests_up_to_the_time_budget():
+    w = synth.scaled(synth.WORKLOADS["tiny"], B=3)
+    sids = synth.workload_catalog(w)
+    one = bench.cpu_baseline_logits(w, sids, "full", 0.0, min_s=0.0)  # at least one request
+    assert one["kind"] == "oracle" and one["cores"] == 1 and one["value"] > 0
+    assert "requests 0..0 of tiny (1 of B=3)" in one["sample"]
+    every = bench.cpu_baseline_logits(w, sids, "full", 0.0, min_s=1e9)  # at most B requests
+    assert "requests 0..2 of tiny (3 of B=3)" in every["sample"]
+
+
+def test_cpu_baseline_lmhead_takes_rows_four_at_a_time():
+    w = synth.WORKLOADS["tiny"]
+    rng = np.random.default_rng(0)
+    weight = rng.integers(-128, 128, size=(w.V, 16)).astype(np.float32) / 8192.0
+    rows = rng.integers(-128, 128, size=(10, 16)).astype(np.float32) / 64.0
+    cb = bench.cpu_baseline_lmhead(w, rows, weight, min_s=1e9)
+    assert cb["kind"] == "oracle" and cb["value"] > 0
+    assert "for 10 rows of request 0" in cb["sample"]
+    assert "(%d rows: 1 at step 0" % (1 + (w.depth - 1) * w.K) in cb["sample"]
