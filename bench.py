@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="with --config serving: skip the records of the other catalog-scale workloads")
     p.add_argument("--ref-requests", type=int, default=1, help="requests per reference-arm sample")
     p.add_argument("--batch", type=int, default=0, help="override B (requests per GPU), e.g. for profiling")
     p.add_argument("--norm", default="full", choices=["full", "sid_range", "candidates"],
@@ -288,7 +290,7 @@ def cpu_baseline_logits(w: synth.Workload, sids: np.ndarray, norm: str, temperat
         method += smp["method_s"]
         gen += smp["gen_s"]
         n += 1
-    return {"value": cand / method, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": cand / method, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_description(),
             "sample": "requests 0..%d of %s (%d of B=%d), a full decode each, single-threaded C oracle in double, "
                       "time excluding its logits generation (%.1f s method, %.1f s generation)"
                       % (n - 1, w.name, n, w.B, method, gen)}
@@ -309,6 +311,7 @@ def cpu_baseline_lmhead(w: synth.Workload, rows: np.ndarray, weight: np.ndarray,
         per_req = smp["rows_per_request"]
     per_row = secs / done
     return {"value": w.K * w.depth / (per_req * per_row), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "host": host_description(),
             "sample": "oracle lm_head rows (hidden . W^T over V = %d, d = %d, in double) for %d rows of "
                       "request 0, %.2f s per row, scaled to one request's decode (%d rows: 1 at step 0, "
                       "K afterwards); the selection's cost is negligible next to the rows"
@@ -361,7 +364,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config,
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                         "host": host_description()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -533,45 +537,37 @@ def run_lmhead(args):
         dist.destroy_process_group()
 
 
-def main():
-    args = parse_args()
-    if args.impl == "reference":
-        run_reference(args)
-        return
-    if args.lmhead:
-        run_lmhead(args)
-        return
+def host_description() -> dict:
+    """The host the CPU legs ran on: logical cores and CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: int, barrier, slowest,
+                            with_e2e: bool) -> dict:
+    """One logits-path workload on this rank's GPU: build the trie (timed on
+    its own), produce every step's logits with an untimed decode, then time
+    `args.steps` whole decodes twice (the headline with nothing recorded
+    between kernels, then with the library's per-kernel events for the
+    roofline and the per-step breakdown), and optionally the end-to-end
+    decode through host buffers.  Frees everything it allocated."""
     import torch
-    import torch.distributed as dist
 
     from trie_constrained_beam_fr_b200 import fr
 
-    rank, world, local_rank = dist_env()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def slowest(x: float) -> float:
-        return max_over_ranks(x, world, dist, dev)
-
-    w = synth.WORKLOADS[args.config]
-    if args.batch:
-        w = synth.scaled(w, B=args.batch)
     B, K, D, V = w.B, w.K, w.depth, w.V
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     elt = w.elt_size
-    b_offset, _ = rank_requests(rank, world, B)  # each rank decodes its own requests
-
     sids_np = synth.workload_catalog(w)
     sids = torch.from_numpy(sids_np).to(dev)
-    stream = torch.cuda.current_stream()
 
     # catalog trie (off the per-decode path; timed on its own)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -583,6 +579,7 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     trie_ms = e0.elapsed_time(e1)
+    del sids
     levels = fr.fr_trie_level_sizes(trie)
     beam = fr.fr_beam_init(trie, B, K, V, w.dtype)
     norm_code = {"full": fr.FR_NORM_FULL, "sid_range": fr.FR_NORM_SID_RANGE,
@@ -591,7 +588,7 @@ def main():
     if args.temperature > 0:
         fr.fr_beam_set_sampling(beam, args.temperature, 0x5EED, b_offset)
     # columns each live row's log-sum-exp streams (none over the candidate slice)
-    row_cols = {"full": V, "sid_range": w.depth * w.C, "candidates": 0}[args.norm]
+    row_cols = {"full": V, "sid_range": sum(w.codebook_sizes), "candidates": 0}[args.norm]
 
     # one untimed decode produces every step's logits (prefix-dependent)
     bufs = [torch.empty((B, K, V), dtype=tdt, device=dev) for _ in range(D)]
@@ -662,18 +659,16 @@ def main():
     alg_bytes = sum(per_step_bytes[i % D] for i in range(n_launch))
     stream_total_ms = float(np.sum(stream_ms))
     achieved = alg_bytes / (stream_total_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w.name)
-    if args.norm != "full":
-        traffic = None  # the committed counters are for the full-vocabulary stream
     row_kernel = ("k_slice_candidates" if not row_cols else
                   "k_rows_short" if row_cols * elt <= 16384 else "k_stream")
-    if row_kernel != "k_stream":
-        traffic = None  # the committed counters are for k_stream
+    # the committed counters are for k_stream over the full vocabulary
+    traffic = recorded_traffic(w.name) if (args.norm == "full" and row_kernel == "k_stream") else None
     roofline = {"bound": "hbm" if row_cols else "latency", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
                 "kernel": row_kernel, "timing": "per-kernel CUDA events, second timed pass of the same decodes",
                 "alg_bytes_per_launch": alg_bytes / max(1, n_launch),
-                "ms_per_launch": stream_total_ms / max(1, n_launch)}
+                "ms_per_launch": stream_total_ms / max(1, n_launch),
+                "frac_of_8tbs": achieved / 8000.0}
     per_step = []
     for t in range(D):
         sm = [stream_ms[i] for i in range(t, n_launch, D)]
@@ -685,7 +680,7 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         host = []
         try:
             for t in range(D):
@@ -725,26 +720,90 @@ def main():
                "ms_per_step": e2e_ms, "steps": args.e2e_steps}
         del host
 
+    fr.fr_beam_destroy(beam)
+    fr.fr_trie_destroy(trie)
+    del bufs, out_sids, out_scores, out_items
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"config": logits_config(w, args, levels), "value": value, "ms_per_step": ms_per_decode,
+            "hbm_gbs": hbm_gbs_decode, "hbm_frac_of_8tbs": hbm_gbs_decode / 8000.0,
+            "ms_per_step_with_kernel_events": evented_ms / args.steps, "roofline": roofline,
+            "per_step": per_step, "trie_build_ms": trie_ms, "clocks": clocks.summary(), "e2e": e2e,
+            "sids_np": sids_np}
+
+
+# The catalog-scale workloads recorded beside the serving headline.
+OTHER_CATALOG_WORKLOADS = ["wide_deep", "narrow", "skewed"]
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    if args.lmhead:
+        run_lmhead(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, world, dist, dev)
+
+    def workload(name: str) -> synth.Workload:
+        w = synth.WORKLOADS[name]
+        return synth.scaled(w, B=args.batch) if args.batch else w
+
+    w = workload(args.config)
+    b_offset, _ = rank_requests(rank, world, w.B)  # each rank decodes its own requests
+    head = measure_logits_workload(w, args, dev, world, b_offset, barrier, slowest, with_e2e=not args.no_e2e)
+    sids_np = head.pop("sids_np")
+
+    # the other catalog-scale workloads at full size (same timing, no e2e /
+    # CPU leg), each one's buffers freed before the next
+    others = {}
+    if args.config == "serving" and not args.no_workloads:
+        for name in OTHER_CATALOG_WORKLOADS:
+            wo = workload(name)
+            bo, _ = rank_requests(rank, world, wo.B)
+            r = measure_logits_workload(wo, args, dev, world, bo, barrier, slowest, with_e2e=False)
+            r.pop("sids_np")
+            r.pop("e2e")
+            r["gpu_launches"] = args.steps * (2 * wo.depth + 2)
+            others[name] = r
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_logits(w, sids_np, args.norm, args.temperature)
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_decode, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": logits_config(w, args, levels),
-            "hbm_gbs": hbm_gbs_decode, "hbm_frac_of_8tbs": hbm_gbs_decode / 8000.0,
-            "ms_per_step_with_kernel_events": evented_ms / args.steps,
-            "roofline": roofline, "per_step": per_step, "trie_build_ms": trie_ms,
-            "gpu_launches": args.steps * (2 * D + 2),
-            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu,
+            "config": head["config"],
+            "hbm_gbs": head["hbm_gbs"], "hbm_frac_of_8tbs": head["hbm_frac_of_8tbs"],
+            "ms_per_step_with_kernel_events": head["ms_per_step_with_kernel_events"],
+            "roofline": head["roofline"], "per_step": head["per_step"], "trie_build_ms": head["trie_build_ms"],
+            "gpu_launches": args.steps * (2 * w.depth + 2),
+            "clocks": head["clocks"], "e2e": head["e2e"], "cpu_baseline": cpu,
         }
+        if others:
+            line["workloads"] = others
         print(json.dumps(line), flush=True)
-    fr.fr_beam_destroy(beam)
-    fr.fr_trie_destroy(trie)
     if world > 1:
         dist.destroy_process_group()
 

@@ -290,12 +290,19 @@ void fr_beam_destroy(fr_beam* beam);
  *   rows        1 .. 65536 (the scratch's capacity; more -> FR_ERR_INVALID_ARG)
  *   lse_dev     device float [rows], written
  * Asynchronous on `stream`.  The first call on a device looks up the
- * scratch's device address (once per device, with that device current); make
- * that first call before any stream capture.  All calls share the one
- * scratch array and leave their contents in it: calls whose work can overlap
- * on the GPU (different streams, or different host threads) race and must be
- * serialised by the caller.  A row holding NaN or +inf gets a non-finite
- * result; no status word is kept. */
+ * scratch's device address and raises the kernel's shared-memory limit (once
+ * per device, with that device current); make that first call before any
+ * stream capture.  That lookup is cached per device ordinal, so the entry
+ * point must not be used again after cudaDeviceReset.  All calls share the
+ * one scratch array and leave their contents in it: calls whose work can
+ * overlap on the GPU (different streams, or different host threads) race and
+ * must be serialised by the caller.  Every call first sets lse_dev[0..rows)
+ * to NaN.  A row holding NaN or +inf gets a non-finite result, and so does
+ * every row the kernel could not finish because one of its bounded waits
+ * (2 s) ran out; no status word is kept, so a non-finite lse is the only
+ * error signal from the device.  Host-side argument errors return
+ * FR_ERR_INVALID_ARG before any work is queued; a failed launch returns
+ * FR_ERR_CUDA. */
 fr_status fr_row_logsumexp_noalloc(const void* logits_dev, int64_t ld, fr_dtype dtype, int32_t rows, int32_t V,
                                    float* lse_dev, fr_stream stream);
 

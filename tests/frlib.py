@@ -1,18 +1,35 @@
 """Helpers shared by the GPU parity tests: drive the CUDA library through its C
 ABI and compare its results with the oracle's under the near-tie protocol.
 
-Protocol (scores are fp32 on the GPU, double in the oracle; tolerance 1e-4):
-  * the live counts are equal;
+Protocol at temperature 0 (scores are fp32 on the GPU, double in the oracle;
+tolerance 1e-4; the order is the strict total order of "beamgrad 2.0.0
+PKG-INFO", §Features: score descending, then parent slot, then token):
+  * the live counts are equal and the dead slots are marked;
   * rank by rank, |score_gpu - score_oracle| <= 1e-4 (order statistics move by
     at most the largest perturbation, so rank-wise comparison is sound);
+  * the GPU's survivors are distinct (parent, token) pairs, its scores do not
+    increase, and survivors with bitwise-equal fp32 scores come in ascending
+    (parent, token) order;
   * wherever the oracle's score at rank j is separated by more than 1e-4 from
     its neighbours (rank j-1 above, rank j+1 or the best excluded candidate
-    below), parent slot and token are identical.
+    below), parent slot and token are identical;
+  * inside a near-tie group (a run of ranks whose neighbouring oracle scores
+    are within 1e-4) every GPU survivor is one of the oracle's survivors of
+    that group, with that candidate's oracle score within 1e-4; where the group
+    reaches the best excluded candidate (the K-th place), a GPU survivor
+    outside the oracle's group must be a real candidate whose oracle score is
+    within 1e-4 of the GPU's score for it (the oracle's whole candidate list,
+    from a step with K widened to every candidate);
+  * where the oracle's scores tie exactly at the K-th place (more candidates
+    with the same double score than slots left) and those candidates share one
+    parent -- so both sides compute bitwise-equal scores for them -- the GPU
+    keeps exactly the oracle's survivors, lowest tokens first.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass
-from typing import List, Optional
+import dataclasses
+from dataclasses import dataclass, field
+from typing import Callable, Dict, List, Optional, Tuple
 
 import numpy as np
 import torch
@@ -119,28 +136,159 @@ class GpuBeam:
         return fr.fr_beam_set_state(self.beam, t, live, prefix, score, kv)
 
 
+@dataclass
+class TieStats:
+    """What the near-tie checks of compare_step covered."""
+    steps: int = 0
+    near_tie_ranks: int = 0      # ranks inside near-tie groups (membership checked)
+    exact_tie_ranks: int = 0     # ranks inside runs of bitwise-equal GPU scores (order checked)
+    boundary_exact: int = 0      # exact ties straddling the K-th place, GPU survivors checked one for one
+    boundary_swaps: int = 0      # GPU survivors outside the oracle's boundary group, verified as candidates
+    unverified: int = 0          # boundary members that could not be verified (no candidate list)
+
+    def summary(self) -> str:
+        return ("%d steps: %d near-tie ranks, %d exact-tie ranks, %d exact ties at the K-th place, "
+                "%d verified boundary swaps, %d unverified"
+                % (self.steps, self.near_tie_ranks, self.exact_tie_ranks, self.boundary_exact,
+                   self.boundary_swaps, self.unverified))
+
+
+class OracleCands:
+    """Every candidate of one request at step t, from the oracle's state after
+    step t - 1 (the root at t = 0): (parent slot, token) -> oracle score
+    (double).  The oracle's own step with K widened to the candidate count
+    keeps them all.  Computed lazily and cached; hash and constant logits only
+    (the lm_head mode indexes hidden states by K)."""
+
+    def __init__(self, cfg, cat, b: int, ref=None, b_ref: Optional[int] = None):
+        self.cfg, self.cat, self.b, self.ref = cfg, cat, b, ref
+        self.b_ref = b if b_ref is None else b_ref
+        self._cache: Dict[int, Dict[Tuple[int, int], float]] = {}
+
+    def state(self, t: int):
+        K, D = self.cfg.K, self.cfg.depth
+        if t == 0:
+            prefix = np.full((K, D), -1, np.int32)
+            score = np.full(K, -np.inf)
+            score[0] = 0.0
+            return 1, prefix, score
+        r = self.ref
+        return int(r.step_live[t - 1, self.b_ref]), r.step_prefix[t - 1, self.b_ref], r.step_score[t - 1, self.b_ref]
+
+    def at(self, t: int) -> Dict[Tuple[int, int], float]:
+        if t not in self._cache:
+            live, prefix, score = self.state(t)
+            K, D = self.cfg.K, self.cfg.depth
+            wide = dataclasses.replace(self.cfg, K=max(K, live * int(self.cfg.codebook[t])))
+            pre = np.full((wide.K, D), -1, np.int32)
+            pre[:K] = prefix
+            sc = np.full(wide.K, -np.inf)
+            sc[:K] = score
+            r = oracle.step(wide, self.cat, self.b, t, live, pre, sc)
+            self._cache[t] = {(int(r.parent[j]), int(r.token[j])): float(r.score[j]) for j in range(r.live)}
+        return self._cache[t]
+
+
 def compare_step(gpu_live, gpu_parent, gpu_token, gpu_score, or_live, or_parent, or_token, or_score,
-                 or_excluded, where: str = "") -> List[str]:
-    """Near-tie protocol for one request's step.  Returns a list of problems
-    (empty when the step matches)."""
+                 or_excluded, where: str = "", cands: Optional[Callable[[], Dict]] = None,
+                 stats: Optional[TieStats] = None) -> List[str]:
+    """Near-tie protocol for one request's step (module docstring).  `cands`,
+    if given, returns the oracle's whole candidate list of the step
+    (OracleCands.at); `stats` accumulates what was checked.  Returns a list of
+    problems (empty when the step matches)."""
+    st = stats if stats is not None else TieStats()
+    st.steps += 1
     bad = []
     if int(gpu_live) != int(or_live):
         return ["%s live %d != oracle %d" % (where, gpu_live, or_live)]
     n = int(or_live)
-    d = np.abs(gpu_score[:n].astype(np.float64) - or_score[:n])
+    gp = [(int(gpu_parent[j]), int(gpu_token[j])) for j in range(n)]
+    op = [(int(or_parent[j]), int(or_token[j])) for j in range(n)]
+    gs = np.asarray(gpu_score[:n], dtype=np.float32)
+    os_ = np.asarray(or_score[:n], dtype=np.float64)
+    d = np.abs(gs.astype(np.float64) - os_)
     if n and d.max() > TOL:
         j = int(d.argmax())
-        bad.append("%s score rank %d: gpu %.7f oracle %.7f" % (where, j, gpu_score[j], or_score[j]))
-    for j in range(n):
-        above = j == 0 or or_score[j - 1] - or_score[j] > TOL
-        below_score = or_score[j + 1] if j + 1 < n else or_excluded
-        below = (not np.isfinite(below_score)) or or_score[j] - below_score > TOL
-        if above and below and (gpu_parent[j] != or_parent[j] or gpu_token[j] != or_token[j]):
-            bad.append("%s rank %d: gpu (parent %d, token %d) oracle (%d, %d), score %.7f"
-                       % (where, j, gpu_parent[j], gpu_token[j], or_parent[j], or_token[j], or_score[j]))
+        bad.append("%s score rank %d: gpu %.7f oracle %.7f" % (where, j, gs[j], os_[j]))
     if np.any(gpu_parent[n:] != -1) or np.any(gpu_token[n:] != -1) or np.any(np.isfinite(gpu_score[n:])):
         bad.append("%s dead slots not marked" % where)
+    if len(set(gp)) != n:
+        bad.append("%s survivors not distinct" % where)
+    # the GPU's own order: scores non-increasing, bitwise-equal scores in
+    # ascending (parent, token) order
+    for j in range(n - 1):
+        if gs[j] < gs[j + 1]:
+            bad.append("%s ranks %d, %d out of score order" % (where, j, j + 1))
+        elif gs[j] == gs[j + 1]:
+            st.exact_tie_ranks += 1
+            if gp[j] >= gp[j + 1]:
+                bad.append("%s ranks %d, %d: equal scores but (parent, token) %s before %s"
+                           % (where, j, j + 1, gp[j], gp[j + 1]))
+    boundary = float(or_excluded)
+    j = 0
+    while j < n:
+        hi = j
+        while hi + 1 < n and os_[hi] - os_[hi + 1] <= TOL:
+            hi += 1
+        reaches = bool(np.isfinite(boundary)) and os_[hi] - boundary <= TOL
+        if hi == j and not reaches:
+            if gp[j] != op[j]:
+                bad.append("%s rank %d: gpu (parent %d, token %d) oracle (%d, %d), score %.7f"
+                           % (where, j, gp[j][0], gp[j][1], op[j][0], op[j][1], os_[j]))
+            j = hi + 1
+            continue
+        st.near_tie_ranks += hi - j + 1
+        group = {op[i]: float(os_[i]) for i in range(j, hi + 1)}
+        outside = sum(1 for r in range(j, hi + 1) if gp[r] not in group)
+        for r in range(j, hi + 1):
+            g = gp[r]
+            if g in group:
+                if abs(float(gs[r]) - group[g]) > TOL:
+                    bad.append("%s near-tie rank %d: %s score gpu %.7f oracle %.7f" % (where, r, g, gs[r], group[g]))
+                continue
+            if not reaches:
+                bad.append("%s near-tie rank %d: gpu %s not in the oracle's group" % (where, r, g))
+                continue
+            if cands is None:
+                st.unverified += 1
+                continue
+            c = cands()
+            if g not in c:
+                bad.append("%s boundary rank %d: gpu %s is not a candidate" % (where, r, g))
+            elif abs(c[g] - float(gs[r])) > TOL:
+                bad.append("%s boundary rank %d: gpu %s score %.7f, oracle's score of it %.7f"
+                           % (where, r, g, gs[r], c[g]))
+            else:
+                st.boundary_swaps += 1
+        # exact ties at the K-th place: more candidates share the last
+        # survivor's double score than slots are left
+        if reaches and boundary == os_[hi] and cands is not None:
+            a = hi
+            while a > j and os_[a - 1] == os_[hi]:
+                a -= 1
+            tied = sorted(g for g, v in cands().items() if v == os_[hi])
+            if len({g[0] for g in tied}) == 1:
+                # one parent, one logit value: bitwise-equal GPU scores, so the
+                # GPU keeps a lowest-token prefix of them (all the oracle
+                # keeps, unless a near-tied candidate of another parent took a
+                # slot, which the membership checks above verified)
+                st.boundary_exact += 1
+                tset = set(tied)
+                kept = sorted(g for g in gp if g in tset)
+                if kept != tied[: len(kept)] or len(kept) < hi - a + 1 - outside:
+                    bad.append("%s exact tie at the K-th place (ranks %d..%d, %d tied candidates of parent %d): "
+                               "gpu keeps %s, lowest tokens %s" % (where, a, hi, len(tied), tied[0][0], kept,
+                                                                   tied[: hi - a + 1]))
+        j = hi + 1
     return bad
+
+
+def diverged(gpu_parent, gpu_token, or_parent, or_token, n: int) -> bool:
+    """The GPU kept other (valid, near-tied) survivors or another order than
+    the oracle: a free-running decode continues from another state, so later
+    steps are not comparable."""
+    n = int(n)
+    return bool(np.any(gpu_parent[:n] != or_parent[:n]) or np.any(gpu_token[:n] != or_token[:n]))
 
 
 def key_tol(temperature: float) -> float:
@@ -202,12 +350,6 @@ def check_key_order(gpu_live, gpu_parent, gpu_token, gpu_score, temperature: flo
     tol = key_tol(temperature)
     return ["%s keys out of order at rank %d: %.7f < %.7f" % (where, j, k[j], k[j + 1])
             for j in range(n - 1) if k[j] < k[j + 1] - tol]
-
-
-def near_tie_in(or_score, or_live, or_excluded) -> bool:
-    n = int(or_live)
-    s = list(or_score[:n]) + ([or_excluded] if np.isfinite(or_excluded) else [])
-    return any(s[i] - s[i + 1] <= TOL for i in range(len(s) - 1))
 
 
 def check_invariants(w: synth.Workload, sids_np: np.ndarray, gpu_sids, gpu_scores, gpu_items, live,

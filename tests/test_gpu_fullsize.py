@@ -7,13 +7,15 @@ independent, so the oracle decodes them one at a time -- are checked step by
 step under teacher forcing: the full batch is set to the GPU's own state except
 the sampled requests, which get the oracle's state, and one GPU step must then
 match the oracle's next step under the near-tie protocol."""
+import functools
+
 import numpy as np
 import pytest
 
 import oracle
 from trie_constrained_beam_fr_b200 import synth
 
-from frlib import GpuBeam, check_invariants, compare_step, near_tie_in, oracle_cfg
+from frlib import GpuBeam, OracleCands, TieStats, check_invariants, compare_step, diverged, oracle_cfg
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -24,26 +26,35 @@ def test_full_size_workload(name):
     sids = synth.workload_catalog(w)
     samples = [0, w.B - 1]
     cat = oracle.Catalog(sids, w.codebook_sizes)
-    refs = {b: oracle.decode(oracle_cfg(w, B=1, b_offset=b), cat) for b in samples}
+    cfgs = {b: oracle_cfg(w, B=1, b_offset=b) for b in samples}
+    refs = {b: oracle.decode(cfgs[b], cat) for b in samples}
+    # each sampled request's whole candidate list per step (request index 0
+    # of a one-request oracle whose offset is b), computed only when a tie
+    # reaches the K-th place
+    cands = {b: OracleCands(cfgs[b], cat, 0, refs[b]) for b in samples}
+    stats = TieStats()
     gpu = GpuBeam(w, sids)
     try:
         views = gpu.decode()
         g_sids, g_scores, g_items = gpu.finalize()
         check_invariants(w, sids, g_sids, g_scores, g_items, views[-1].live)
 
-        # free running, sampled requests
+        # free running, sampled requests (compared until the GPU keeps other
+        # valid near-tied survivors, after which the decodes differ)
+        problems = []
         for b in samples:
             r = refs[b]
             for t in range(w.depth):
-                p = compare_step(views[t].live[b], views[t].parent[b], views[t].token[b], views[t].score[b],
-                                 r.step_live[t, 0], r.step_parent[t, 0], r.step_token[t, 0], r.step_score[t, 0],
-                                 r.step_excluded[t, 0], where="free t=%d b=%d" % (t, b))
-                if p:
-                    assert near_tie_in(r.step_score[t, 0], r.step_live[t, 0], r.step_excluded[t, 0]), p
+                problems += compare_step(views[t].live[b], views[t].parent[b], views[t].token[b],
+                                         views[t].score[b], r.step_live[t, 0], r.step_parent[t, 0],
+                                         r.step_token[t, 0], r.step_score[t, 0], r.step_excluded[t, 0],
+                                         where="free t=%d b=%d" % (t, b), cands=functools.partial(cands[b].at, t),
+                                         stats=stats)
+                if diverged(views[t].parent[b], views[t].token[b], r.step_parent[t, 0], r.step_token[t, 0],
+                            r.step_live[t, 0]):
                     break
 
         # teacher forced, sampled requests, full batch
-        problems = []
         for t in range(w.depth):
             if t == 0:
                 live = np.ones(w.B, np.int32)
@@ -65,7 +76,9 @@ def test_full_size_workload(name):
                 r = refs[b]
                 problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], r.step_live[t, 0],
                                          r.step_parent[t, 0], r.step_token[t, 0], r.step_score[t, 0],
-                                         r.step_excluded[t, 0], where="forced t=%d b=%d" % (t, b))
+                                         r.step_excluded[t, 0], where="forced t=%d b=%d" % (t, b),
+                                         cands=functools.partial(cands[b].at, t), stats=stats)
         assert not problems, "\n".join(problems[:20])
+        print("%s: %s" % (name, stats.summary()))
     finally:
         gpu.close()

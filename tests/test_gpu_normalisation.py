@@ -3,13 +3,15 @@ oracle: the SID token range ("flashrec 0.1.1 METADATA", §Features/Decoding:
 the projection covers only the ids of the SID tokens) and the candidate slice
 ("Qwen-2.5-1B-RLCD-Fast", §Parallel Evaluation step 4).  Same near-tie
 protocol and tolerance as the full-vocabulary tests."""
+import functools
+
 import numpy as np
 import pytest
 
 import oracle
 from trie_constrained_beam_fr_b200 import fr, synth
 
-from frlib import GpuBeam, check_invariants, compare_step, near_tie_in, oracle_cfg
+from frlib import GpuBeam, OracleCands, check_invariants, compare_step, diverged, oracle_cfg
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +36,9 @@ def test_teacher_forced_and_free_running(name, norm):
     w = CASES[name]
     sids = synth.workload_catalog(w)
     cat = oracle.Catalog(sids, w.codebook_sizes)
-    ref = oracle.decode(oracle_cfg(w, norm=norm), cat)
+    cfg = oracle_cfg(w, norm=norm)
+    ref = oracle.decode(cfg, cat)
+    cands = {b: OracleCands(cfg, cat, b, ref) for b in range(w.B)}
     gpu = GpuBeam(w, sids, norm=norm)
     problems = []
     try:
@@ -54,7 +58,8 @@ def test_teacher_forced_and_free_running(name, norm):
             for b in range(B):
                 problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], ref.step_live[t, b],
                                          ref.step_parent[t, b], ref.step_token[t, b], ref.step_score[t, b],
-                                         ref.step_excluded[t, b], where="forced t=%d b=%d" % (t, b))
+                                         ref.step_excluded[t, b], where="forced t=%d b=%d" % (t, b),
+                                         cands=functools.partial(cands[b].at, t))
         views = gpu.decode()
         g_sids, g_scores, g_items = gpu.finalize()
     finally:
@@ -65,9 +70,11 @@ def test_teacher_forced_and_free_running(name, norm):
         for t in range(w.depth):
             p = compare_step(views[t].live[b], views[t].parent[b], views[t].token[b], views[t].score[b],
                              ref.step_live[t, b], ref.step_parent[t, b], ref.step_token[t, b],
-                             ref.step_score[t, b], ref.step_excluded[t, b], where="free t=%d b=%d" % (t, b))
-            if p:
-                assert near_tie_in(ref.step_score[t, b], ref.step_live[t, b], ref.step_excluded[t, b]), p
+                             ref.step_score[t, b], ref.step_excluded[t, b], where="free t=%d b=%d" % (t, b),
+                             cands=functools.partial(cands[b].at, t))
+            assert not p, p
+            if diverged(views[t].parent[b], views[t].token[b], ref.step_parent[t, b], ref.step_token[t, b],
+                        ref.step_live[t, b]):
                 break
 
 

@@ -41,9 +41,14 @@ std::mutex g_setup_mutex;
 NoallocScratch* g_scratch_addr[MAX_DEVICES] = {};
 int32_t g_sm_count[MAX_DEVICES] = {};
 
-__global__ void k_noalloc_prepare(NoallocScratch* s, int32_t rows) {
-    // counters of the rows this call uses start at zero; the rest is unused
-    for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x) s->row_cnt[i] = 0;
+__global__ void k_noalloc_prepare(NoallocScratch* s, int32_t rows, float* lse_out) {
+    // counters of the rows this call uses start at zero (the rest is unused);
+    // every output starts as NaN, so a row the streaming kernel never finishes
+    // (a bounded wait that ran out) reads as non-finite, not as stale data
+    for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x) {
+        s->row_cnt[i] = 0;
+        lse_out[i] = __int_as_float(0x7FC00000);
+    }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         s->live = rows;
         s->err = 0;
@@ -52,7 +57,10 @@ __global__ void k_noalloc_prepare(NoallocScratch* s, int32_t rows) {
 
 // Device address of the scratch for the current device, looked up once per
 // device (cudaGetSymbolAddress must run with that device current; in host
-// code the array's name is only a host-side stand-in).
+// code the array's name is only a host-side stand-in), together with the
+// device's SM count and the streaming kernel's shared-memory attribute.  The
+// cache is per device ordinal: after cudaDeviceReset the module may load at
+// another address, so the entry point is not for use across a device reset.
 fr_status scratch_for_current_device(NoallocScratch** out, int32_t* sms) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
@@ -68,6 +76,11 @@ fr_status scratch_for_current_device(NoallocScratch** out, int32_t* sms) {
         }
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+            (void)cudaGetLastError();
+            return FR_ERR_CUDA;
+        }
+        // the streaming kernel's shared-memory limit, raised once per device
+        if (fr::row_lse_kernel_setup() != cudaSuccess) {
             (void)cudaGetLastError();
             return FR_ERR_CUDA;
         }
@@ -94,7 +107,7 @@ extern "C" fr_status fr_row_logsumexp_noalloc(const void* logits_dev, int64_t ld
     if (st != FR_OK) return st;
     const int32_t grid = sms < NOALLOC_MAX_CTAS ? sms : NOALLOC_MAX_CTAS;
     const cudaStream_t cs = (cudaStream_t)stream;
-    k_noalloc_prepare<<<(rows + 255) / 256 < 148 ? (rows + 255) / 256 : 148, 256, 0, cs>>>(s, rows);
+    k_noalloc_prepare<<<(rows + 255) / 256 < sms ? (rows + 255) / 256 : sms, 256, 0, cs>>>(s, rows, lse_dev);
     FR_CUDA_TRY(cudaGetLastError());
     FR_CUDA_TRY(fr::launch_row_lse(logits_dev, ld, (int32_t)dtype, rows, V, grid, &s->live, s->partial, s->row_cnt,
                                    &s->err, lse_dev, cs));

@@ -44,10 +44,7 @@
 namespace fr {
 namespace {
 
-#ifndef FR_NCW
-#define FR_NCW 16
-#endif
-constexpr int NCW = FR_NCW;  // consumer warps: reduce the staged chunks
+constexpr int NCW = 16;  // consumer warps: reduce the staged chunks
 constexpr int NFW = 2;       // finisher warps: lse, cross-CTA combine, candidate scores
 constexpr int PRODUCER_WARP = NCW;
 constexpr int FIRST_FINISHER_WARP = NCW + 1;
@@ -72,12 +69,6 @@ constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
 static_assert(PSLOTS > 2 * MAX_STAGES, "partial slots must outnumber the segments in flight");
 constexpr int64_t GRAN = 1024;  // CTA ranges start at multiples of this many elements
 constexpr float L2E = 1.4426950408889634f;
-#ifndef FR_POLY_PAIRS
-#define FR_POLY_PAIRS 0
-#endif
-// Of the four bf16 pairs in each 16-byte vector, this many take exp2 on the
-// FMA pipe (polynomial) instead of the MUFU.
-constexpr int POLY_PAIRS = FR_POLY_PAIRS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 
@@ -283,11 +274,6 @@ __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
     asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
-__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
-    f32x2 r;
-    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
 __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
     f32x2 r;
     asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -299,36 +285,9 @@ __device__ __forceinline__ f32x2 ex2_pair(f32x2 v) {
     return pack2(ex2_approx(lo), ex2_approx(hi));
 }
 
-// 2^y for a pair on the FMA pipe instead of the MUFU: Cody-Waite reduction
-// y = n + f, n = round(y), f in [-1/2, 1/2], then a degree-5 minimax
-// polynomial for 2^f (relative error 1.5e-7 after rounding the coefficients
-// to float32; coefficients from gen_exp2_poly.py, a Remez fit), then n is
-// added to the exponent field.  Valid for finite y <= 126; y is clamped below
-// at -125, where 2^y is negligible next to any sum it joins.
-__device__ __forceinline__ f32x2 exp2_poly_pair(f32x2 y) {
-    constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-    float y0, y1;
-    unpack2(y, y0, y1);
-    const f32x2 yc = pack2(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
-    const f32x2 t = add2(yc, pack2(MAGIC, MAGIC));       // low mantissa bits hold n
-    const f32x2 f = sub2(yc, sub2(t, pack2(MAGIC, MAGIC)));  // exact
-    f32x2 p = fma2(pack2(1.327647245e-03f, 1.327647245e-03f), f, pack2(9.675540961e-03f, 9.675540961e-03f));
-    p = fma2(p, f, pack2(5.550713092e-02f, 5.550713092e-02f));
-    p = fma2(p, f, pack2(2.402212024e-01f, 2.402212024e-01f));
-    p = fma2(p, f, pack2(6.931469440e-01f, 6.931469440e-01f));
-    p = fma2(p, f, pack2(1.000000119e+00f, 1.000000119e+00f));
-    float p0, p1, t0, t1;
-    unpack2(p, p0, p1);
-    unpack2(t, t0, t1);
-    // bits(t) = bits(MAGIC) + n and bits(MAGIC) << 23 == 0 (mod 2^32), so
-    // bits(t) << 23 == n << 23: the exponent increment.
-    return pack2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
 // Exponent sum of this lane's VPL vectors against the reference point mref:
 // sum 2^(x*log2(e) - mref*log2(e)), in packed pairs.
-template <bool BF16, int POLY, int VPL>
+template <bool BF16, int VPL>
 __device__ __forceinline__ f32x2 lane_expsum(const uint4 (&q)[VPL], float mref) {
     const float nmL = (mref == -INFINITY) ? 0.f : -mref * L2E;
     const f32x2 c2 = pack2(nmL, nmL);
@@ -342,7 +301,7 @@ __device__ __forceinline__ f32x2 lane_expsum(const uint4 (&q)[VPL], float mref) 
             for (int e = 0; e < 4; ++e) {
                 const f32x2 x = pack2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
                 const f32x2 y = fma2(x, l2, c2);
-                acc[e] = add2(acc[e], (e < POLY) ? exp2_poly_pair(y) : ex2_pair(y));
+                acc[e] = add2(acc[e], ex2_pair(y));
             }
         } else {
             const f32x2 x0 = pack2(__uint_as_float(w[0]), __uint_as_float(w[1]));
@@ -408,7 +367,7 @@ template <bool BF16, int VPL>
 __device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f32x2& s2) {
     float mref = m;
     if (mref == -INFINITY) mref = BF16 ? __uint_as_float(q[0].x << 16) : __uint_as_float(q[0].x);
-    f32x2 part = lane_expsum<BF16, BF16 ? POLY_PAIRS : 0>(q, mref);
+    f32x2 part = lane_expsum<BF16>(q, mref);
     float plo, phi;
     unpack2(part, plo, phi);
     if (!(mref > -INFINITY && plo + phi <= 0x1p64f)) {
@@ -418,7 +377,7 @@ __device__ __forceinline__ void lane_consume(const uint4 (&q)[VPL], float& m, f3
             const float sc = ex2_approx((m - mn) * L2E);
             s2 = mul2(s2, pack2(sc, sc));
         }
-        part = lane_expsum<BF16, 0>(q, mn);
+        part = lane_expsum<BF16>(q, mn);
         mref = mn;
     }
     s2 = add2(s2, part);
@@ -813,7 +772,7 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
             s2 = mul2(s2, pack2(sc, sc));
         }
         m = mn;
-        if (m != -INFINITY) s2 = add2(s2, lane_expsum<BF16, 0>(q, m));
+        if (m != -INFINITY) s2 = add2(s2, lane_expsum<BF16>(q, m));
     }
     for (int64_t i = lane; i < a0; i += 32) lane_add(m, s2, load_elem(sg.ptr, i, ELT));
     for (int64_t i = a1 + lane; i < W; i += 32) lane_add(m, s2, load_elem(sg.ptr, i, ELT));
@@ -1006,13 +965,18 @@ cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const T
     return cudaLaunchKernelEx(&L.cfg, k_rows_given_lse, a);
 }
 
+cudaError_t row_lse_kernel_setup() {
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)stream_smem_bytes(1, true));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_stream<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)stream_smem_bytes(1, false));
+}
+
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
                            const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
                            cudaStream_t s) {
     const int max_bytes = (int)stream_smem_bytes(1, dtype == FR_BF16);
-    cudaError_t e = cudaFuncSetAttribute(dtype == FR_BF16 ? k_stream<true, true> : k_stream<false, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, max_bytes);
-    if (e != cudaSuccess) return e;
     StreamArgs a{};
     a.logits = static_cast<const char*>(logits);
     a.ld = ld;

@@ -81,6 +81,9 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
 // Log-sum-exp of `rows` rows (row k at logits + k*ld elements) into lse_out,
 // with caller-provided scratch: partial [2*grid], row_cnt [rows] (zero on
 // entry, zero again on exit), err [1]; live_dev [1] must hold `rows`.
+// row_lse_kernel_setup raises the kernel's shared-memory limit on the current
+// device; it must have run there once before launch_row_lse.
+cudaError_t row_lse_kernel_setup();
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
                            const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
                            cudaStream_t s);

@@ -320,11 +320,29 @@ def fr_beam_destroy(beam) -> None:
 
 def fr_row_logsumexp_noalloc(logits: torch.Tensor, rows: int, V: int, lse: torch.Tensor,
                              ld: Optional[int] = None, stream=None) -> None:
-    """Allocation-free log-sum-exp of `rows` logits rows (see include/fr.h)."""
+    """Allocation-free log-sum-exp of `rows` logits rows (see include/fr.h).
+
+    Row k is `V` elements at element offset k * ld from the start of
+    `logits`.  Every row must lie inside the tensor's storage and `lse` must
+    hold `rows` values, both on the current CUDA device: the C side cannot
+    see tensor bounds, so these are checked here before the launch."""
     if lse.dtype != torch.float32 or not lse.is_cuda:
         raise ValueError("lse must be a float32 CUDA tensor")
+    if not logits.is_cuda:
+        raise ValueError("logits must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if logits.device.index != cur or lse.device.index != cur:
+        raise ValueError("logits and lse must be on the current CUDA device (%d)" % cur)
     if ld is None:
         ld = logits.stride(-2) if logits.dim() >= 2 else V
+    rows, V, ld = int(rows), int(V), int(ld)
+    if rows < 1 or V < 1 or ld < V:
+        raise ValueError("need rows >= 1, V >= 1 and ld >= V")
+    if lse.numel() < rows or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous and hold at least `rows` values")
+    avail = logits.untyped_storage().nbytes() // logits.element_size() - logits.storage_offset()
+    if (rows - 1) * ld + V > avail:
+        raise ValueError("rows x ld reach past the end of the logits tensor's storage")
     _check(libfr().fr_row_logsumexp_noalloc(_dev_ptr(logits), int(ld), _dtype_code(logits.dtype), int(rows),
                                             int(V), _dev_ptr(lse), _stream(stream)), "fr_row_logsumexp_noalloc")
 
