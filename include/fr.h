@@ -202,6 +202,9 @@ fr_status fr_lmhead_init(const void* weight_dev, int64_t ldw, int32_t V, int32_t
 fr_status fr_lmhead_run(fr_lmhead* lmhead, const void* hidden_dev, int64_t ldh, int32_t rows, float* lse_dev,
                         float* slice_dev, fr_stream stream);
 fr_status fr_lmhead_status(fr_lmhead* lmhead);
+/* Clears the handle's sticky device status (stream-ordered, asynchronous), so
+ * that the handle can be used again after an error was read. */
+fr_status fr_lmhead_clear_status(fr_lmhead* lmhead, fr_stream stream);
 void fr_lmhead_destroy(fr_lmhead* lmhead);
 
 /* One beam step from given rows instead of logits (the lm_head path, §8 f1:
@@ -274,6 +277,28 @@ fr_status fr_beam_read_timing(fr_beam* beam, float* stream_ms, float* select_ms,
                               int32_t* n);
 
 void fr_beam_destroy(fr_beam* beam);
+
+/* ------------------------------------------------------------------------ */
+/* Test hooks for the failure path (no counterpart in the pages).  Every wait
+ * a kernel makes on an mbarrier or on a flag set by another warp is bounded:
+ * when the limit passes, the kernel records FR_ERR_DEVICE in the handle's
+ * sticky status, stops issuing work, lets the copies and tensor-core
+ * operations it already issued complete, frees its tensor memory and
+ * returns, leaving the CUDA context usable.  These calls let a test make such
+ * a wait expire on purpose, without any fault:
+ *   wait_limit_ns  limit of those waits, 1,000 .. 60,000,000,000 ns, or 0 for
+ *                  the default (2 s)
+ *   starve_copies  1: the producer warp of the streaming kernel (for a beam)
+ *                  or of the lm_head kernel issues no copies at all, so the
+ *                  consumers' first wait cannot complete and expires after
+ *                  wait_limit_ns; 0: normal operation
+ * Host-side settings that apply from the next fr_beam_step /
+ * fr_lmhead_run; FR_ERR_INVALID_ARG for a NULL handle or values outside the
+ * ranges above.  With starve_copies = 1 the step's outputs are meaningless;
+ * fr_beam_reset (or fr_lmhead_clear_status) after setting 0 restores normal
+ * operation. */
+fr_status fr_beam_set_wait_test(fr_beam* beam, uint64_t wait_limit_ns, int32_t starve_copies);
+fr_status fr_lmhead_set_wait_test(fr_lmhead* lmhead, uint64_t wait_limit_ns, int32_t starve_copies);
 
 /* ------------------------------------------------------------------------ */
 /* Allocation-free row log-sum-exp.  No counterpart in the pages: this is a

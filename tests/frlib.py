@@ -28,7 +28,8 @@ PKG-INFO", §Features: score descending, then parent slot, then token):
 from __future__ import annotations
 
 import dataclasses
-from dataclasses import dataclass, field
+import functools
+from dataclasses import dataclass
 from typing import Callable, Dict, List, Optional, Tuple
 
 import numpy as np
@@ -289,6 +290,30 @@ def diverged(gpu_parent, gpu_token, or_parent, or_token, n: int) -> bool:
     steps are not comparable."""
     n = int(n)
     return bool(np.any(gpu_parent[:n] != or_parent[:n]) or np.any(gpu_token[:n] != or_token[:n]))
+
+
+def free_running_problems(w, gpu_views, g_sids, g_items, ref, cfg, cat) -> List[str]:
+    """Full decodes compared step by step; after a step where the GPU kept
+    other valid near-tied survivors (or another order), the two decodes go on
+    from different states and are not compared further."""
+    cands = {b: OracleCands(cfg, cat, b, ref) for b in range(w.B)}
+    problems = []
+    for b in range(w.B):
+        same = True
+        for t in range(w.depth):
+            v = gpu_views[t]
+            problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], ref.step_live[t, b],
+                                     ref.step_parent[t, b], ref.step_token[t, b], ref.step_score[t, b],
+                                     ref.step_excluded[t, b], where="free t=%d b=%d" % (t, b),
+                                     cands=functools.partial(cands[b].at, t))
+            if diverged(v.parent[b], v.token[b], ref.step_parent[t, b], ref.step_token[t, b], ref.step_live[t, b]):
+                same = False
+                break
+        if same and g_sids is not None:
+            n = int(ref.step_live[-1, b])
+            np.testing.assert_array_equal(g_sids[b, :n], ref.sids[b, :n])
+            np.testing.assert_array_equal(g_items[b, :n], ref.items[b, :n])
+    return problems
 
 
 def key_tol(temperature: float) -> float:

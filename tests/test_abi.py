@@ -91,6 +91,9 @@ def test_every_handle_call_rejects_a_null_handle_without_a_gpu():
     assert L.fr_beam_read_timing(None, None, None, 0, ctypes.byref(i32)) == bad
     assert L.fr_lmhead_run(None, ctypes.c_void_p(16), 64, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), None) == bad
     assert L.fr_lmhead_status(None) == bad
+    assert L.fr_lmhead_clear_status(None, None) == bad
+    assert L.fr_beam_set_wait_test(None, 1000000, 1) == bad
+    assert L.fr_lmhead_set_wait_test(None, 1000000, 1) == bad
     L.fr_trie_destroy(None)
     L.fr_beam_destroy(None)
     L.fr_lmhead_destroy(None)

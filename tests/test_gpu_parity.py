@@ -12,7 +12,8 @@ import pytest
 import oracle
 from trie_constrained_beam_fr_b200 import synth
 
-from frlib import GpuBeam, OracleCands, TieStats, check_invariants, compare_step, diverged, oracle_cfg
+from frlib import (GpuBeam, OracleCands, TieStats, check_invariants, compare_step, diverged,
+                   free_running_problems, oracle_cfg)
 
 pytestmark = pytest.mark.gpu
 
@@ -141,30 +142,6 @@ def test_teacher_forced_steps(name):
         assert stats.boundary_exact >= TIE_CASES[name], stats.summary()
 
 
-def _free_running(w, sids, gpu_views, g_sids, g_items, ref, cfg, cat):
-    """Full decodes compared step by step; after a step where the GPU kept
-    other valid near-tied survivors (or another order), the two decodes go on
-    from different states and are not compared further."""
-    cands = {b: OracleCands(cfg, cat, b, ref) for b in range(w.B)}
-    problems = []
-    for b in range(w.B):
-        same = True
-        for t in range(w.depth):
-            v = gpu_views[t]
-            problems += compare_step(v.live[b], v.parent[b], v.token[b], v.score[b], ref.step_live[t, b],
-                                     ref.step_parent[t, b], ref.step_token[t, b], ref.step_score[t, b],
-                                     ref.step_excluded[t, b], where="free t=%d b=%d" % (t, b),
-                                     cands=functools.partial(cands[b].at, t))
-            if diverged(v.parent[b], v.token[b], ref.step_parent[t, b], ref.step_token[t, b], ref.step_live[t, b]):
-                same = False
-                break
-        if same and g_sids is not None:
-            n = int(ref.step_live[-1, b])
-            np.testing.assert_array_equal(g_sids[b, :n], ref.sids[b, :n])
-            np.testing.assert_array_equal(g_items[b, :n], ref.items[b, :n])
-    return problems
-
-
 @pytest.mark.parametrize("name", list(SMALL))
 def test_free_running_decode(name):
     w = SMALL[name]
@@ -179,7 +156,7 @@ def test_free_running_decode(name):
     finally:
         gpu.close()
     check_invariants(w, sids, g_sids, g_scores, g_items, views[-1].live)
-    problems = _free_running(w, sids, views, g_sids, g_items, ref, cfg, cat)
+    problems = free_running_problems(w, views, g_sids, g_items, ref, cfg, cat)
     assert not problems, "\n".join(problems[:20])
 
 
@@ -243,7 +220,7 @@ def test_strided_and_unaligned_rows(misalign, ld_pad, name):
     finally:
         gpu.close()
     cfg = oracle_cfg(w)
-    problems = _free_running(w, sids, views, None, None, ref, cfg, oracle.Catalog(sids, w.codebook_sizes))
+    problems = free_running_problems(w, views, None, None, ref, cfg, oracle.Catalog(sids, w.codebook_sizes))
     assert not problems, "\n".join(problems[:20])
 
 

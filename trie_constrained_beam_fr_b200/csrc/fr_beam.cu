@@ -93,6 +93,8 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bm->shape.grid = sms;
     bm->shape.norm = FR_NORM_FULL;
     bm->shape.sid_span = (int32_t)(span - trie->sid_base);
+    bm->shape.wait_ns = FR_WAIT_LIMIT_NS;
+    bm->shape.starve = 0;
     for (int t = 0; t < D; ++t) {
         // step t: live beams (1 at the root, then at most K) times the level's fan-out
         const int64_t bound = (int64_t)(t == 0 ? 1 : K) * std::max(1, trie->level_fanout[t]);
@@ -325,6 +327,15 @@ extern "C" fr_status fr_beam_set_sampling(fr_beam* bm, float temperature, uint64
     bm->shape.inv_temp = inv;
     bm->shape.gseed = seed;
     bm->shape.req_offset = request_offset;
+    return FR_OK;
+}
+
+extern "C" fr_status fr_beam_set_wait_test(fr_beam* bm, uint64_t wait_limit_ns, int32_t starve_copies) {
+    if (!bm || (wait_limit_ns != 0 && (wait_limit_ns < 1000ull || wait_limit_ns > 60000000000ull)) ||
+        (starve_copies != 0 && starve_copies != 1))
+        return FR_ERR_INVALID_ARG;
+    bm->shape.wait_ns = wait_limit_ns ? wait_limit_ns : FR_WAIT_LIMIT_NS;
+    bm->shape.starve = starve_copies;
     return FR_OK;
 }
 

@@ -13,6 +13,10 @@
 // Device status word values (sticky; the first error wins).
 #define FR_DEV_OK 0
 
+// Limit of every bounded device-side wait (on an mbarrier or on a flag another
+// warp sets), unless a test setting shortens it.
+#define FR_WAIT_LIMIT_NS 2000000000ull
+
 namespace fr {
 
 // Device view of a built trie, passed to kernels by value.

@@ -23,9 +23,9 @@
 //              slice, then release the accumulator to the next tile.
 //   k_lmhead_combine   one warp per row: lse = M + ln sum_t s_t e^(m_t - M).
 //
-// Every mbarrier wait is bounded (2 s): on expiry the kernel records
-// FR_ERR_DEVICE, stops issuing, waits (bounded) for the copies and MMAs it
-// issued, frees its tensor memory and returns.
+// Every mbarrier wait is bounded (2 s, or the limit a test setting gives): on
+// expiry the kernel records FR_ERR_DEVICE, stops issuing, waits (bounded) for
+// the copies and MMAs it issued, frees its tensor memory and returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -49,7 +49,6 @@ constexpr int LM_THREADS = 256;           // 8 warps
 constexpr int LM_A_BYTES = LM_BM * LM_BK * 2;  // 16 KB
 constexpr int LM_B_BYTES = LM_BN * LM_BK * 2;  // 32 KB
 constexpr int LM_TMEM_COLS = 2 * LM_BN;        // two accumulators
-constexpr uint64_t LM_WAIT_NS = 2000000000ull;
 constexpr float LM_L2E = 1.4426950408889634f;
 
 static_assert(LM_BK * 2 == 128, "one K stage is one 128-byte swizzle span");
@@ -100,13 +99,13 @@ __device__ __forceinline__ uint64_t lm_now_ns() {
 
 // Bounded wait; false after the time limit or once another thread aborted.
 __device__ __forceinline__ bool lm_wait(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
-                                        int32_t* err) {
+                                        int32_t* err, uint64_t limit_ns) {
     if (lm_mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = lm_now_ns();
     for (uint32_t it = 0;; ++it) {
         if (lm_mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if ((it & 63u) == 63u && lm_now_ns() - t0 > LM_WAIT_NS) {
+        if ((it & 63u) == 63u && lm_now_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             set_error(err, FR_ERR_DEVICE);
             return false;
@@ -119,7 +118,7 @@ __device__ __forceinline__ void lm_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = lm_now_ns();
     for (uint32_t it = 0;; ++it) {
         if (lm_mbar_try_wait(bar, parity)) return;
-        if ((it & 63u) == 63u && lm_now_ns() - t0 > LM_WAIT_NS) return;
+        if ((it & 63u) == 63u && lm_now_ns() - t0 > FR_WAIT_LIMIT_NS) return;
     }
 }
 
@@ -191,6 +190,8 @@ struct LmArgs {
     float2* partial;  // [rows, n_tiles] (max, sum of e^(x - max))
     float* slice;     // [rows, sid_span]
     int32_t* err;
+    uint64_t wait_ns;  // limit of the bounded waits that give up (abort)
+    int32_t starve;    // test setting: the producer issues no TMA loads, so the MMA thread's waits expire
 };
 
 struct LmSmem {
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(LM_THREADS, 1)
     const uint32_t tmem = sm->tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !a.starve) {
             // producer: one (tile, k-block) after another through the ring
             uint32_t it = 0;
             bool ok = true;
@@ -250,7 +251,8 @@ __global__ void __launch_bounds__(LM_THREADS, 1)
                 const int m0 = (tile % a.m_tiles) * LM_BM, n0 = (tile / a.m_tiles) * LM_BN;
                 for (int kb = 0; kb < k_blocks; ++kb, ++it) {
                     const int s = (int)(it % LM_STAGES);
-                    if (it >= (uint32_t)LM_STAGES && !lm_wait(&sm->empty[s], ((it / LM_STAGES) & 1u) ^ 1u, abort_flag, a.err)) {
+                    if (it >= (uint32_t)LM_STAGES &&
+                        !lm_wait(&sm->empty[s], ((it / LM_STAGES) & 1u) ^ 1u, abort_flag, a.err, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(LM_THREADS, 1)
             bool ok = true;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++local) {
                 const int acc = local & 1;
-                if (local >= 2 && !lm_wait(&sm->tmem_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag, a.err)) {
+                if (local >= 2 && !lm_wait(&sm->tmem_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag, a.err, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(LM_THREADS, 1)
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * LM_BN);
                 for (int kb = 0; kb < k_blocks; ++kb, ++it) {
                     const int s = (int)(it % LM_STAGES);
-                    if (!lm_wait(&sm->full[s], (it / LM_STAGES) & 1u, abort_flag, a.err)) {
+                    if (!lm_wait(&sm->full[s], (it / LM_STAGES) & 1u, abort_flag, a.err, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(LM_THREADS, 1)
         int local = 0;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
             const int acc = local & 1;
-            if (!lm_wait(&sm->tmem_full[acc], (local >> 1) & 1, abort_flag, a.err)) break;
+            if (!lm_wait(&sm->tmem_full[acc], (local >> 1) & 1, abort_flag, a.err, a.wait_ns)) break;
             lm_fence_after();
             const int mt = tile % a.m_tiles, nt = tile / a.m_tiles;
             const int row = mt * LM_BM + r_in, n0 = nt * LM_BN;
@@ -438,6 +440,8 @@ struct fr_lmhead {
     float2* partial = nullptr;  // [max_rows, n_tiles]
     int32_t* err = nullptr;
     cudaStream_t last_stream = nullptr;
+    uint64_t wait_ns = FR_WAIT_LIMIT_NS;
+    int32_t starve = 0;
 };
 
 extern "C" fr_status fr_lmhead_init(const void* weight_dev, int64_t ldw, int32_t V, int32_t d, int32_t max_rows,
@@ -504,6 +508,8 @@ extern "C" fr_status fr_lmhead_run(fr_lmhead* h, const void* hidden_dev, int64_t
     a.partial = h->partial;
     a.slice = slice_dev;
     a.err = h->err;
+    a.wait_ns = h->wait_ns;
+    a.starve = h->starve;
     const int tiles = a.m_tiles * a.n_tiles;
     const int grid = std::min(tiles, h->sms);
     fr::k_lmhead<<<grid, fr::LM_THREADS, fr::lm_smem_bytes(), s>>>(map_h, h->map_w, a);
@@ -519,6 +525,23 @@ extern "C" fr_status fr_lmhead_status(fr_lmhead* h) {
     int32_t err = 0;
     FR_CUDA_TRY(cudaMemcpy(&err, h->err, sizeof(int32_t), cudaMemcpyDeviceToHost));
     return (fr_status)err;
+}
+
+extern "C" fr_status fr_lmhead_clear_status(fr_lmhead* h, fr_stream stream) {
+    if (!h) return FR_ERR_INVALID_ARG;
+    const cudaStream_t s = (cudaStream_t)stream;
+    FR_CUDA_TRY(cudaMemsetAsync(h->err, 0, sizeof(int32_t), s));
+    h->last_stream = s;
+    return FR_OK;
+}
+
+extern "C" fr_status fr_lmhead_set_wait_test(fr_lmhead* h, uint64_t wait_limit_ns, int32_t starve_copies) {
+    if (!h || (wait_limit_ns != 0 && (wait_limit_ns < 1000ull || wait_limit_ns > 60000000000ull)) ||
+        (starve_copies != 0 && starve_copies != 1))
+        return FR_ERR_INVALID_ARG;
+    h->wait_ns = wait_limit_ns ? wait_limit_ns : FR_WAIT_LIMIT_NS;
+    h->starve = starve_copies;
+    return FR_OK;
 }
 
 extern "C" void fr_lmhead_destroy(fr_lmhead* h) {

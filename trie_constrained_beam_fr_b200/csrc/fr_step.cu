@@ -32,8 +32,9 @@
 // counter-based SplitMix64 stream indexed by (request, step, parent slot,
 // token), for the selection to rank.
 //
-// Every wait on an mbarrier is bounded: after 2 s the kernel records
-// FR_ERR_DEVICE in the beam's status word and returns.
+// Every wait on an mbarrier or on a flag is bounded: after 2 s (or the limit
+// a test setting gives) the kernel records FR_ERR_DEVICE in the beam's status
+// word and returns, with no copy in flight.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -69,7 +70,6 @@ constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
 static_assert(PSLOTS > 2 * MAX_STAGES, "partial slots must outnumber the segments in flight");
 constexpr int64_t GRAN = 1024;  // CTA ranges start at multiples of this many elements
 constexpr float L2E = 1.4426950408889634f;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 
 
@@ -114,6 +114,8 @@ struct StreamArgs {
     float inv_temp;      // 1 / temperature
     uint64_t gseed;      // seed of the Gumbel stream
     int64_t req_offset;  // index of local request 0 in the Gumbel stream
+    uint64_t wait_ns;    // limit of the bounded waits that give up (abort)
+    int32_t starve;      // test setting: the producer issues no copies, so the consumers' waits expire
 };
 
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the finaliser of a Weyl
@@ -153,13 +155,13 @@ struct Seg {
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
-                                         int32_t* err) {
+                                         int32_t* err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             set_error(err, FR_ERR_DEVICE);
             return false;
@@ -172,21 +174,21 @@ __device__ __forceinline__ void wait_bar_drain(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) return;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > FR_WAIT_LIMIT_NS) return;
     }
 }
 
 // Bounded wait until *word == want (a sequence number written by another warp
 // of this CTA).  Returns false on abort or after the time limit.
 __device__ __forceinline__ bool wait_seq(volatile int32_t* word, int32_t want, volatile int32_t* abort_flag,
-                                         int32_t* err) {
+                                         int32_t* err, uint64_t limit_ns) {
     if (*word == want) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (*word == want) return true;
         if (*abort_flag) return false;
         __nanosleep(64);
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             set_error(err, FR_ERR_DEVICE);
             return false;
@@ -574,7 +576,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
     const int64_t r_first = bg / a.W, r_last = (eg - 1) / a.W;
 
     if (warp == PRODUCER_WARP) {
-        if (lane == 0) {
+        if (lane == 0 && !a.starve) {
             uint32_t chunk = 0;
             int st = 0;
             uint32_t ph = 0;
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
                 const char* src = sg.ptr + sg.a0 * ELT;
                 int64_t left = (sg.a1 - sg.a0) * ELT;
                 for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
-                    if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err)) {
+                    if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -619,7 +621,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
         const int64_t njobs = r_last - r_first + 1;
         for (int64_t j = warp - FIRST_FINISHER_WARP; j < njobs; j += NFW) {
             const int slot = (int)(j % QCAP);
-            if (!wait_seq(&hdr->ready[slot], (int32_t)(j + 1), &hdr->abort_flag, a.err)) return;
+            if (!wait_seq(&hdr->ready[slot], (int32_t)(j + 1), &hdr->abort_flag, a.err, a.wait_ns)) return;
             __threadfence_block();
             const Job job = hdr->jobs[slot];
             __syncwarp();
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
         const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
         const int32_t nvec_all = (int32_t)((sg.a1 - sg.a0) * ELT / 16);
         for (int j = 0; j < sg.nchunks; ++j) {
-            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err)) return;
+            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err, a.wait_ns)) return;
             if (j == 0 && cw == 0 && lane < sg.a0 - sg.c0) lane_add(m, s2, load_elem(sg.ptr, sg.c0 + lane, ELT));
             const uint4* stage = reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES);
             const int32_t nvec = min(nvec_all - j * VEC_PER_STAGE, VEC_PER_STAGE);
@@ -700,7 +702,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
                 if (lane == 0) hdr->segcnt[ps] = 0;
                 const int slot = (int)(jid % QCAP);
                 if (jid >= QCAP &&
-                    !wait_seq(&hdr->freed[slot], (int32_t)(jid - QCAP + 1), &hdr->abort_flag, a.err))
+                    !wait_seq(&hdr->freed[slot], (int32_t)(jid - QCAP + 1), &hdr->abort_flag, a.err, a.wait_ns))
                     return;
                 if (lane == 0) {
                     hdr->jobs[slot] = Job{r, pm, pv};
@@ -909,6 +911,8 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.inv_temp = sh.inv_temp;
     a.gseed = sh.gseed;
     a.req_offset = sh.req_offset;
+    a.wait_ns = sh.wait_ns ? sh.wait_ns : FR_WAIT_LIMIT_NS;
+    a.starve = sh.starve;
     a.row_stride_b = sh.K;
     a.col_sub = 0;
     a.lse_in = nullptr;
@@ -958,6 +962,7 @@ cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const T
     a.inv_temp = sh.inv_temp;
     a.gseed = sh.gseed;
     a.req_offset = sh.req_offset;
+    a.wait_ns = FR_WAIT_LIMIT_NS;
     const dim3 warp_grid((unsigned)sh.B, (unsigned)((sh.K + 7) / 8));
     StepLaunch L(warp_grid, 256, 0, s);
     if (sh.norm == FR_NORM_CANDIDATES) return cudaLaunchKernelEx(&L.cfg, k_slice_candidates, a);
@@ -992,6 +997,8 @@ cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_
     a.row_cnt = row_cnt;
     a.err = err;
     a.lse_out = lse_out;
+    a.wait_ns = FR_WAIT_LIMIT_NS;
+    a.starve = 0;
     if (dtype == FR_BF16)
         k_stream<true, true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
     else

@@ -31,6 +31,8 @@ struct StepShape {
     float inv_temp;      // 1 / temperature; 0 = deterministic top-K
     uint64_t gseed;      // Gumbel stream seed
     int64_t req_offset;  // index of local request 0 in the Gumbel stream
+    uint64_t wait_ns;    // limit of the streaming kernel's bounded waits
+    int32_t starve;      // test setting: the streaming kernel's producer issues no copies
 };
 
 // Launch configuration of a step kernel: programmatic stream serialization

@@ -65,10 +65,13 @@ FR_FUNCS = [
     ("fr_beam_set_timing", _I32, [_VP, _I32]),
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
+    ("fr_beam_set_wait_test", _I32, [_VP, _U64, _I32]),
     ("fr_row_logsumexp_noalloc", _I32, [_VP, _I64, _I32, _I32, _I32, _VP, _VP]),
     ("fr_lmhead_init", _I32, [_VP, _I64, _I32, _I32, _I32, _I32, _I32, _P(_VP)]),
     ("fr_lmhead_run", _I32, [_VP, _VP, _I64, _I32, _VP, _VP, _VP]),
     ("fr_lmhead_status", _I32, [_VP]),
+    ("fr_lmhead_clear_status", _I32, [_VP, _VP]),
+    ("fr_lmhead_set_wait_test", _I32, [_VP, _U64, _I32]),
     ("fr_lmhead_destroy", None, [_VP]),
 ]
 FR_GEN_FUNCS = [
@@ -301,6 +304,13 @@ def fr_beam_set_sampling(beam, temperature: float, seed: int = 0, request_offset
                                         int(request_offset)), "fr_beam_set_sampling")
 
 
+def fr_beam_set_wait_test(beam, wait_limit_ns: int = 0, starve_copies: bool = False) -> None:
+    """Test hook: shorten the streaming kernel's bounded waits and make its
+    producer issue no copies, so that a wait expires (see include/fr.h)."""
+    _check(libfr().fr_beam_set_wait_test(beam, int(wait_limit_ns), int(bool(starve_copies))),
+           "fr_beam_set_wait_test")
+
+
 def fr_beam_set_timing(beam, enable: bool) -> None:
     _check(libfr().fr_beam_set_timing(beam, int(bool(enable))), "fr_beam_set_timing")
 
@@ -393,6 +403,16 @@ def fr_lmhead_run(lmhead, hidden: torch.Tensor, lse: torch.Tensor, slice_: Optio
 
 def fr_lmhead_status(lmhead) -> int:
     return int(libfr().fr_lmhead_status(lmhead))
+
+
+def fr_lmhead_clear_status(lmhead, stream=None) -> None:
+    _check(libfr().fr_lmhead_clear_status(lmhead, _stream(stream)), "fr_lmhead_clear_status")
+
+
+def fr_lmhead_set_wait_test(lmhead, wait_limit_ns: int = 0, starve_copies: bool = False) -> None:
+    """Test hook: as fr_beam_set_wait_test, for the lm_head kernel."""
+    _check(libfr().fr_lmhead_set_wait_test(lmhead, int(wait_limit_ns), int(bool(starve_copies))),
+           "fr_lmhead_set_wait_test")
 
 
 def fr_lmhead_destroy(lmhead) -> None:
