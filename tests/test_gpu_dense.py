@@ -13,7 +13,7 @@ import torch
 import oracle
 from trie_constrained_beam_fr_b200 import fr, synth
 
-from frlib import GpuBeam, oracle_cfg
+from frlib import GpuBeam, TieStats, oracle_cfg
 import test_gpu_parity as tp
 
 pytestmark = pytest.mark.gpu
@@ -99,11 +99,13 @@ def test_full_product_catalog_matches_the_oracle(dense):
     """All levels dense, teacher forced (set_state walks the prefixes through
     the direct lookups too)."""
     w, sids = CASES["full_product"]
-    ref = oracle.decode(oracle_cfg(w), oracle.Catalog(sids, w.codebook_sizes))
+    cfg = oracle_cfg(w)
+    cat = oracle.Catalog(sids, w.codebook_sizes)
+    ref = oracle.decode(cfg, cat)
     gpu = GpuBeam(w, sids)
     try:
         fr.fr_trie_set_dense(gpu.trie, dense)
-        problems = tp._teacher_forced(w, sids, gpu, ref)
+        problems = tp._teacher_forced(w, gpu, ref, cfg, cat, TieStats())
     finally:
         gpu.close()
     assert not problems, "\n".join(problems[:20])
