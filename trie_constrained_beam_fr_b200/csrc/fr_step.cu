@@ -16,8 +16,8 @@
 //            1024-element-aligned ranges, one per CTA, so every CTA streams
 //            the same number of bytes whatever the row count.  Inside a CTA
 //            one producer lane moves chunks from HBM into a shared-memory
-//            ring (bf16: 4 stages of 48 KB; fp32: 3 of 56 KB) with 1-D bulk
-//            async copies completing on mbarriers; 16 consumer warps each
+//            ring (bf16: 5 stages of 40 KB; fp32: 3 of 50 KB) with 1-D bulk
+//            async copies completing on mbarriers; 20 consumer warps each
 //            reduce a lane-interleaved slice of every chunk (running
 //            reference + scaled exp2 sum per lane).  At the end of a
 //            row segment the last consumer warp to arrive combines the 16
@@ -45,25 +45,33 @@
 namespace fr {
 namespace {
 
-constexpr int NCW = 16;  // consumer warps: reduce the staged chunks
-constexpr int NFW = 2;       // finisher warps: lse, cross-CTA combine, candidate scores
+// Consumer warps reduce the staged chunks.  The bf16 reduction is bound by
+// the latency of its exponentials (one MUFU ex2 per element), not by their
+// throughput or by HBM: 20 warps hide it better than 16 (measured on B200,
+// serving shape: 5.76 against 5.39-5.69 TB/s), while 22 or 24 warps run out
+// of registers and moving a share of the exponentials to an FMA-pipe
+// polynomial (12.5-50%) was slower at every share.
+constexpr int NCW = 20;
+constexpr int NFW = 2;  // finisher warps: lse, cross-CTA combine, candidate scores
 constexpr int PRODUCER_WARP = NCW;
 constexpr int FIRST_FINISHER_WARP = NCW + 1;
 constexpr int STREAM_THREADS = (NCW + 1 + NFW) * 32;
 // The shared-memory ring of the streaming kernel, per element size (measured
-// on B200 over 3-7 stages of 32-64 KB: bf16 rows stream fastest through 4
-// stages of 48 KB, fp32 rows through 3 of 56 KB; larger chunks amortise the
-// per-chunk barrier work, and bf16 does twice the exponent work per byte).
+// on B200 over 3-7 stages of 32-64 KB: with 20 consumer warps bf16 rows
+// stream fastest through 5 stages of 40 KB, fp32 rows, which are HBM-bound,
+// through 3 of 50 KB; larger chunks amortise the per-chunk barrier work, and
+// bf16 does twice the exponent work per byte).  A stage splits evenly into
+// 16-byte vectors over the consumer lanes.
 template <bool BF16>
 struct Ring {
-    static constexpr int STAGES = BF16 ? 4 : 3;
-    static constexpr int STAGE_BYTES = BF16 ? 49152 : 57344;
+    static constexpr int STAGES = BF16 ? 5 : 3;
+    static constexpr int STAGE_BYTES = BF16 ? 40960 : 51200;
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
     static constexpr int VEC_PER_STAGE = STAGE_BYTES / 16;
     static constexpr int VPL = VEC_PER_STAGE / (NCW * 32);  // 16-byte vectors per lane per chunk
     static_assert(VPL * NCW * 32 == VEC_PER_STAGE, "chunk must split evenly over the consumer lanes");
 };
-constexpr int MAX_STAGES = 4;
+constexpr int MAX_STAGES = 5;
 static_assert(Ring<true>::STAGES <= MAX_STAGES && Ring<false>::STAGES <= MAX_STAGES, "ring stages");
 constexpr int QCAP = 32;    // finished-segment jobs in flight per CTA
 constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
@@ -465,11 +473,11 @@ __device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse) {
 }
 
 // The row's (max, scaled sum) are known: its log-sum-exp, then its
-// candidates (or, LSE_ONLY, just the log-sum-exp).
-template <bool LSE_ONLY>
+// candidates (or, when the log-sum-exps are the output, just the
+// log-sum-exp: row k's at lse_out[k]).
 __device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
     const float lse = m + logf(s);
-    if constexpr (LSE_ONLY) {
+    if (a.lse_out) {
         if ((threadIdx.x & 31) == 0) a.lse_out[sg.k] = lse;
         return;
     }
@@ -477,14 +485,13 @@ __device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, f
 }
 
 // Called by the warp that combined this CTA's partial for row r.
-template <bool LSE_ONLY>
 __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
                                float s) {
     const int lane = threadIdx.x & 31;
     const int64_t fc = (r * a.W) / Q;
     const int64_t lc = ((r + 1) * a.W - 1) / Q;
     if (fc == lc) {
-        finish_row<LSE_ONLY>(a, sg, m, s);
+        finish_row(a, sg, m, s);
         return;
     }
     const int side = (r == r_first) ? 0 : 1;
@@ -511,11 +518,12 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
         combine(M, S, pm, ps);
     }
     if (lane == 0) a.row_cnt[r] = 0;
-    finish_row<LSE_ONLY>(a, sg, M, S);
+    finish_row(a, sg, M, S);
 }
 
-// LSE_ONLY: the rows' log-sum-exps are the output (no trie, no candidates).
-template <bool BF16, bool LSE_ONLY>
+// With a.lse_out set, the rows' log-sum-exps are the output (no trie, no
+// candidates).
+template <bool BF16>
 __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a) {
     constexpr int ELT = BF16 ? 2 : 4;
     constexpr int STAGES = Ring<BF16>::STAGES;
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
                 *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(j + 1);
             }
             const Seg sg = make_seg<ELT>(a, row_start, job.r, bg, eg);
-            finish_segment<LSE_ONLY>(a, sg, job.r, r_first, Q, job.m, job.s);
+            finish_segment(a, sg, job.r, r_first, Q, job.m, job.s);
         }
         return;
     }
@@ -782,7 +790,7 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
     unpack2(s2, lo, hi);
     float s = lo + hi;
     warp_combine(m, s);
-    finish_row<false>(a, sg, m, s);
+    finish_row(a, sg, m, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -876,10 +884,10 @@ size_t stream_smem_bytes(int32_t B, bool bf16) {
 }
 
 cudaError_t stream_kernel_setup() {
-    cudaError_t e = cudaFuncSetAttribute(k_stream<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)stream_smem_bytes(FR_MAX_B, true));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_stream<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(k_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)stream_smem_bytes(FR_MAX_B, false));
 }
 
@@ -927,8 +935,8 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
                                    : cudaLaunchKernelEx(&L.cfg, k_rows_short<false>, a);
     }
     StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B, sh.dtype == FR_BF16), s);
-    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true, false>, a)
-                               : cudaLaunchKernelEx(&L.cfg, k_stream<false, false>, a);
+    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true>, a)
+                               : cudaLaunchKernelEx(&L.cfg, k_stream<false>, a);
 }
 
 cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
@@ -970,13 +978,7 @@ cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const T
     return cudaLaunchKernelEx(&L.cfg, k_rows_given_lse, a);
 }
 
-cudaError_t row_lse_kernel_setup() {
-    cudaError_t e = cudaFuncSetAttribute(k_stream<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)stream_smem_bytes(1, true));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_stream<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)stream_smem_bytes(1, false));
-}
+cudaError_t row_lse_kernel_setup() { return stream_kernel_setup(); }
 
 cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_t rows, int32_t V, int32_t grid,
                            const int32_t* live_dev, float2* partial, int32_t* row_cnt, int32_t* err, float* lse_out,
@@ -1000,9 +1002,9 @@ cudaError_t launch_row_lse(const void* logits, int64_t ld, int32_t dtype, int32_
     a.wait_ns = FR_WAIT_LIMIT_NS;
     a.starve = 0;
     if (dtype == FR_BF16)
-        k_stream<true, true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
+        k_stream<true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
     else
-        k_stream<false, true><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
+        k_stream<false><<<grid, STREAM_THREADS, (size_t)max_bytes, s>>>(a);
     return cudaGetLastError();
 }
 
