@@ -168,8 +168,27 @@ __device__ void sort_desc_u64(unsigned long long* sel, unsigned long long* buf, 
     __syncthreads();
 }
 
-__device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, int Kp,
-                                 unsigned long long* sel, unsigned long long* scratch) {
+// Per live parent slot k of request b, read before the wait on the row kernel
+// (the previous step's selection or the reset wrote them): its candidates'
+// offset (s_off, live + 1 entries), the first level-(t+1) node of its trie
+// children (s_lo; -1 for a node outside the trie) and its KV slot (s_kv).
+// All threads of the block call it; a __syncthreads must follow before use.
+__device__ __forceinline__ void load_parents(const SelectArgs& a, int b, int live, int32_t* s_off, int32_t* s_lo,
+                                             int32_t* s_kv) {
+    const int K = a.K, t = a.t;
+    for (int i = threadIdx.x; i <= live; i += blockDim.x) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
+    for (int k = threadIdx.x; k < live; k += blockDim.x) {
+        const int64_t ok = (int64_t)b * K + k;
+        const int32_t np = a.cur.node[ok];
+        int32_t lo = -1, hi = -1;
+        if (np >= 0 && np < a.trie.nodes[t]) trie_children(a.trie, t, np, lo, hi);
+        s_lo[k] = lo;
+        s_kv[k] = a.cur.kv[ok];
+    }
+}
+
+__device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, const int32_t* s_lo,
+                                 const int32_t* s_kv, int Kp, unsigned long long* sel, unsigned long long* scratch) {
     const int tid = threadIdx.x;
     const int K = a.K, D = a.D, t = a.t;
     sort_desc_u64(sel, scratch, Kp);
@@ -190,12 +209,9 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
             }
             const int k = lo;
             const int64_t ok = (int64_t)b * K + k;
-            const int32_t np = a.cur.node[ok];
             int32_t tok = -1;
-            if (np >= 0 && np < a.trie.nodes[t]) {
-                int32_t lo, hi;
-                trie_children(a.trie, t, np, lo, hi);
-                child = lo + (slot - s_off[k]);
+            if (s_lo[k] >= 0) {
+                child = s_lo[k] + (slot - s_off[k]);
                 if (child >= 0 && child < a.trie.nodes[t + 1]) {
                     tok = a.trie.tok_base[t] + trie_child_code(a.trie, t, child);
                 } else {
@@ -205,7 +221,7 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
             if (child < 0) set_error(a.err, FR_ERR_DEVICE);
             a.nxt.node[oj] = child;
             a.nxt.score[oj] = (a.rank == a.cand) ? key_to_float(key) : a.cand[(int64_t)b * a.cand_stride + slot];
-            a.nxt.kv[oj] = a.cur.kv[ok];
+            a.nxt.kv[oj] = s_kv[k];
             a.parent_out[oj] = k;
             a.token_out[oj] = tok;
             for (int l = 0; l < D; ++l)
@@ -528,17 +544,21 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
 }
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
-    griddep_wait();
-    griddep_launch_dependents();
     __shared__ int32_t s_off[FR_MAX_K + 1];
+    __shared__ int32_t s_lo[FR_MAX_K];
+    __shared__ int32_t s_kv[FR_MAX_K];
     __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_misc[8];
     __shared__ uint32_t red[64];
     const int b = blockIdx.x, tid = threadIdx.x;
     const int K = a.K;
+    // the beam state is not written by the row kernel this one follows: read
+    // it while that kernel drains, then wait for its candidates
     const int live = min(max(a.cur.live[b], 0), K);
-    for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
+    load_parents(a, b, live, s_off, s_lo, s_kv);
+    griddep_wait();
+    griddep_launch_dependents();
     __syncthreads();
     int n = s_off[live];
     if (n < 0 || (int64_t)n > a.cand_stride) {
@@ -548,7 +568,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     const int Kp = min(K, n);
     const int got = block_topk<false>(GlobalCands{a.rank + (int64_t)b * a.cand_stride}, n, Kp, sel, hist, red, s_misc);
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+    select_sort_emit(a, b, live, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
 // ---------------------------------------------------------------------------
@@ -574,13 +594,13 @@ size_t csel_smem_bytes(int64_t key_cap, int cs, int K) {
 }
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectArgs a) {
-    griddep_wait();
-    griddep_launch_dependents();
     cg::cluster_group cl = cg::this_cluster();
     extern __shared__ __align__(16) uint32_t keys[];  // this CTA's keys; in the leader, then the pool
     __shared__ __align__(16) int32_t hist[HBINS];    // also the sort's scratch
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_off[FR_MAX_K + 1];
+    __shared__ int32_t s_lo[FR_MAX_K];
+    __shared__ int32_t s_kv[FR_MAX_K];
     __shared__ uint32_t red[64];
     __shared__ int32_t s_misc[8];
     __shared__ int32_t s_cnt;
@@ -589,9 +609,14 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     const int b = blockIdx.x / CS;
     const int tid = threadIdx.x;
     const int K = a.K;
+    // the leader reads the beam state (not written by the row kernel) while
+    // that kernel drains; every CTA then waits for the candidates
     const int live = min(max(a.cur.live[b], 0), K);
     const int32_t* off_row = a.cur.cand_off + (int64_t)b * (K + 1);
+    if (c == 0) load_parents(a, b, live, s_off, s_lo, s_kv);
     int n = off_row[live];
+    griddep_wait();
+    griddep_launch_dependents();
     if (n < 0 || (int64_t)n > a.cand_stride || (n + CS - 1) / CS > a.key_cap) {
         if (tid == 0 && c == 0) set_error(a.err, FR_ERR_DEVICE);
         n = 0;
@@ -600,8 +625,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     const int S = (n + CS - 1) / CS;
     const int lo = min(n, c * S), hi = min(n, lo + S);
     const int cnt = hi - lo;
-    if (c == 0)
-        for (int i = tid; i <= live; i += SEL_THREADS) s_off[i] = off_row[i];
     const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;
     int i0 = tid;
     for (; i0 + 7 * SEL_THREADS < cnt; i0 += 8 * SEL_THREADS) {
@@ -638,7 +661,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     if (c != 0) return;
     const int got = block_topk<false>(PoolVals{pool}, P, min(Kp, P), sel, hist, red, s_misc);
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(a, b, live, s_off, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+    select_sort_emit(a, b, live, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
 
 // ---------------------------------------------------------------------------

@@ -415,37 +415,85 @@ __device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
     }
 }
 
+// A row's candidate writer needs, besides the row's log-sum-exp, the beam's
+// running score, its trie children and its candidate offset, and the
+// children's logits.  None of these depends on the reduction, so the finisher
+// loads them (and the first batch of the children's logits: lane l holds
+// children l, l + 32, ..., l + 32 (GATHER - 1)) before it waits for the row,
+// while the row is still streaming; only the rest of the gathers, for rows
+// with more than 32 * GATHER children, come after.
+constexpr int GATHER = 8;  // independent gathers in flight per lane
+struct RowPrep {
+    float sc;
+    int32_t lo, nch, base;  // nch < 0: the beam's node or offsets are out of range
+    float x[GATHER];
+};
+
+__device__ __forceinline__ RowPrep prep_cands(const StreamArgs& a, const Seg& sg) {
+    RowPrep p;
+    p.sc = 0.f;
+    p.lo = p.base = 0;
+    p.nch = -1;
+#pragma unroll
+    for (int u = 0; u < GATHER; ++u) p.x[u] = 0.f;
+    if (a.lse_out) return p;  // log-sum-exps only: no candidates
+    const int lane = threadIdx.x & 31;
+    const int64_t bk = (int64_t)sg.b * a.K + sg.k;
+    const int t = a.t;
+    const int32_t n = a.node[bk];
+    const int32_t base = a.cand_off[(int64_t)sg.b * (a.K + 1) + sg.k];
+    p.sc = a.score[bk];
+    if (n < 0 || n >= a.trie.nodes[t]) return p;
+    int32_t lo, hi;
+    trie_children(a.trie, t, n, lo, hi);
+    if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) return p;
+    p.lo = lo;
+    p.nch = hi - lo;
+    p.base = base;
+    const int32_t* codes = a.trie.code[t + 1] + lo;
+    const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
+    const int32_t tb = a.trie.tok_base[t] - a.col_sub;
+#pragma unroll
+    for (int u = 0; u < GATHER; ++u) {
+        const int32_t i = u * 32 + lane;
+        if (i < p.nch) p.x[u] = load_elem(sg.row, tb + (dense ? i : __ldg(codes + i)), a.elt);
+    }
+    return p;
+}
+
 // The row's log-sum-exp is known: write the scores of the trie children of
-// the row's beam (token v of the row at column v - col_sub).  One warp.
-__device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse) {
+// the row's beam (token v of the row at column v - col_sub), from what
+// prep_cands loaded.  One warp.
+__device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse, const RowPrep& p) {
     const int lane = threadIdx.x & 31;
     if (!isfinite(lse)) {
         if (lane == 0) set_error(a.err, FR_ERR_NAN_LOGIT);
     }
-    const int64_t bk = (int64_t)sg.b * a.K + sg.k;
+    if (p.nch < 0) {
+        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
+        return;
+    }
     const int t = a.t;
-    const int32_t n = a.node[bk];
-    if (n < 0 || n >= a.trie.nodes[t]) {
-        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
-        return;
-    }
-    int32_t lo, hi;
-    trie_children(a.trie, t, n, lo, hi);
-    const int32_t base = a.cand_off[(int64_t)sg.b * (a.K + 1) + sg.k];
-    if (lo < 0 || hi < lo || base < 0 || (int64_t)base + (hi - lo) > a.cand_stride) {
-        if (lane == 0) set_error(a.err, FR_ERR_DEVICE);
-        return;
-    }
-    const float sc = a.score[bk];
-    const int32_t* codes = a.trie.code[t + 1] + lo;
+    const float sc = p.sc;
+    const int32_t* codes = a.trie.code[t + 1] + p.lo;
     const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
     const int32_t tb = a.trie.tok_base[t];
-    float* out = a.cand + (int64_t)sg.b * a.cand_stride + base;
-    const int32_t nch = hi - lo;
+    float* out = a.cand + (int64_t)sg.b * a.cand_stride + p.base;
+    const int32_t nch = p.nch;
     if (a.cand_key) {
-        float* key = a.cand_key + (int64_t)sg.b * a.cand_stride + base;
+        float* key = a.cand_key + (int64_t)sg.b * a.cand_stride + p.base;
         const uint64_t rh = gumbel_row_hash(a.gseed, a.req_offset + sg.b, t);
-        for (int32_t i = lane; i < nch; i += 32) {
+#pragma unroll
+        for (int u = 0; u < GATHER; ++u) {
+            const int32_t i = u * 32 + lane;
+            if (i < nch) {
+                const int32_t tok = tb + (dense ? i : __ldg(codes + i));
+                const float v = sc + (p.x[u] - lse);
+                out[i] = v;
+                key[i] = v * a.inv_temp + gumbel_noise(rh, sg.k, tok);
+            }
+        }
+        for (int32_t i = 32 * GATHER + lane; i < nch; i += 32) {
             const int32_t tok = tb + (dense ? i : __ldg(codes + i));
             const float v = sc + (load_elem(sg.row, tok - a.col_sub, a.elt) - lse);
             out[i] = v;
@@ -453,19 +501,24 @@ __device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse) {
         }
         return;
     }
-    constexpr int U = 8;  // independent gathers in flight per lane
-    for (int32_t i0 = 0; i0 < nch; i0 += 32 * U) {
-        int32_t code[U];
-        float x[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < GATHER; ++u) {
+        const int32_t i = u * 32 + lane;
+        if (i < nch) out[i] = sc + (p.x[u] - lse);
+    }
+    for (int32_t i0 = 32 * GATHER; i0 < nch; i0 += 32 * GATHER) {
+        int32_t code[GATHER];
+        float x[GATHER];
+#pragma unroll
+        for (int u = 0; u < GATHER; ++u) {
             const int32_t i = i0 + u * 32 + lane;
             code[u] = i < nch ? (dense ? i : __ldg(codes + i)) : -1;
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u] - a.col_sub, a.elt) : 0.f;
+        for (int u = 0; u < GATHER; ++u)
+            x[u] = code[u] >= 0 ? load_elem(sg.row, tb + code[u] - a.col_sub, a.elt) : 0.f;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < GATHER; ++u) {
             const int32_t i = i0 + u * 32 + lane;
             if (i < nch) out[i] = sc + (x[u] - lse);
         }
@@ -475,23 +528,23 @@ __device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse) {
 // The row's (max, scaled sum) are known: its log-sum-exp, then its
 // candidates (or, when the log-sum-exps are the output, just the
 // log-sum-exp: row k's at lse_out[k]).
-__device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s) {
+__device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, float m, float s, const RowPrep& p) {
     const float lse = m + logf(s);
     if (a.lse_out) {
         if ((threadIdx.x & 31) == 0) a.lse_out[sg.k] = lse;
         return;
     }
-    finish_cands(a, sg, lse);
+    finish_cands(a, sg, lse, p);
 }
 
 // Called by the warp that combined this CTA's partial for row r.
 __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
-                               float s) {
+                               float s, const RowPrep& p) {
     const int lane = threadIdx.x & 31;
     const int64_t fc = (r * a.W) / Q;
     const int64_t lc = ((r + 1) * a.W - 1) / Q;
     if (fc == lc) {
-        finish_row(a, sg, m, s);
+        finish_row(a, sg, m, s, p);
         return;
     }
     const int side = (r == r_first) ? 0 : 1;
@@ -518,7 +571,7 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
         combine(M, S, pm, ps);
     }
     if (lane == 0) a.row_cnt[r] = 0;
-    finish_row(a, sg, M, S);
+    finish_row(a, sg, M, S, p);
 }
 
 // With a.lse_out set, the rows' log-sum-exps are the output (no trie, no
@@ -629,6 +682,9 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
         const int64_t njobs = r_last - r_first + 1;
         for (int64_t j = warp - FIRST_FINISHER_WARP; j < njobs; j += NFW) {
             const int slot = (int)(j % QCAP);
+            const int64_t r = r_first + j;
+            const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
+            const RowPrep prep = prep_cands(a, sg);  // while row r streams
             if (!wait_seq(&hdr->ready[slot], (int32_t)(j + 1), &hdr->abort_flag, a.err, a.wait_ns)) return;
             __threadfence_block();
             const Job job = hdr->jobs[slot];
@@ -637,8 +693,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
                 __threadfence_block();
                 *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(j + 1);
             }
-            const Seg sg = make_seg<ELT>(a, row_start, job.r, bg, eg);
-            finish_segment(a, sg, job.r, r_first, Q, job.m, job.s);
+            finish_segment(a, sg, r, r_first, Q, job.m, job.s, prep);
         }
         return;
     }
@@ -763,6 +818,7 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
     const int64_t nvec = (W - a0) / VE;
     const int64_t a1 = a0 + nvec * VE;
     const uint4* vec = reinterpret_cast<const uint4*>(sg.ptr + a0 * ELT);
+    const RowPrep prep = prep_cands(a, sg);  // its loads overlap the row's
     const uint32_t ninf = BF16 ? 0xFF80FF80u : 0xFF800000u;
     const uint4 ninf4 = make_uint4(ninf, ninf, ninf, ninf);
     constexpr int VPL = 4;  // 16-byte vectors per lane per batch (2 KB per warp)
@@ -790,7 +846,7 @@ __global__ void __launch_bounds__(256) k_rows_short(const StreamArgs a) {
     unpack2(s2, lo, hi);
     float s = lo + hi;
     warp_combine(m, s);
-    finish_row(a, sg, m, s);
+    finish_row(a, sg, m, s, prep);
 }
 
 // ---------------------------------------------------------------------------
@@ -815,7 +871,8 @@ __global__ void __launch_bounds__(256) k_rows_given_lse(const StreamArgs a) {
     sg.b = b;
     sg.k = k;
     sg.row = a.logits + r * a.ld * a.elt;
-    finish_cands(a, sg, __ldg(a.lse_in + r));
+    const RowPrep prep = prep_cands(a, sg);
+    finish_cands(a, sg, __ldg(a.lse_in + r), prep);
 }
 
 // ---------------------------------------------------------------------------
