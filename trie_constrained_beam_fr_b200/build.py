@@ -28,7 +28,7 @@ TARGETS = {
     "libfr.so": ["fr_trie.cu", "fr_step.cu", "fr_select.cu", "fr_beam.cu", "fr_noalloc.cu", "fr_lmhead.cu"],
     "libfr_gen.so": ["fr_gen.cu"],
 }
-HEADERS = ["fr_internal.cuh", "fr_handles.h", "fr_step.cuh"]
+HEADERS = ["fr_internal.cuh", "fr_handles.h", "fr_step.cuh", "fr_topk.cuh"]
 
 
 def lib_path(name: str) -> str:

@@ -79,7 +79,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
         delete bm;
         return FR_ERR_CUDA;
     }
-    if (fr::stream_kernel_setup() != cudaSuccess) {
+    if (fr::stream_kernel_setup() != cudaSuccess || fr::root_step_setup() != cudaSuccess) {
         (void)cudaGetLastError();
         delete bm;
         return FR_ERR_CUDA;
@@ -117,6 +117,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bytes += 2 * align256(sizeof(int32_t) * bk);                   // parent, token
     bytes += 2 * align256(sizeof(float) * (size_t)B * cand_stride);  // cand, cand_key
     bytes += align256(sizeof(float2) * (size_t)sms * 2);           // partial
+    bytes += align256(sizeof(float2) * (size_t)B * fr::root_step_max_parts());  // root_partial
     bytes += align256(sizeof(int32_t) * bk);                       // row_cnt
     bytes += align256(sizeof(int32_t));                            // err
     cudaError_t e = cudaMalloc(&bm->block, bytes);
@@ -142,6 +143,7 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bm->buf.cand_key = carve<float>(p, (size_t)B * cand_stride);
     bm->buf.cand_stride = cand_stride;
     bm->buf.partial = carve<float2>(p, (size_t)sms * 2);
+    bm->buf.root_partial = carve<float2>(p, (size_t)B * fr::root_step_max_parts());
     bm->buf.row_cnt = carve<int32_t>(p, bk);
     bm->buf.err = carve<int32_t>(p, 1);
 
@@ -179,9 +181,15 @@ extern "C" fr_status fr_beam_step(fr_beam* bm, const void* logits, int64_t ld, f
             if (!ev[i]) FR_CUDA_TRY(cudaEventCreate(&ev[i]));
         FR_CUDA_TRY(cudaEventRecord(ev[0], s));
     }
-    FR_CUDA_TRY(fr::launch_stream(bm->shape, bm->buf, bm->trie->dev, bm->t, logits, ld, s));
-    if (timed) FR_CUDA_TRY(cudaEventRecord(ev[1], s));
-    FR_CUDA_TRY(fr::launch_select(bm->shape, bm->buf, bm->trie->dev, bm->t, s));
+    if (bm->t == 0 && fr::root_step_fused(bm->shape, bm->trie->dev)) {
+        // the whole first step in one kernel (its time is the row kernel's)
+        FR_CUDA_TRY(fr::launch_root_step(bm->shape, bm->buf, bm->trie->dev, logits, ld, s));
+        if (timed) FR_CUDA_TRY(cudaEventRecord(ev[1], s));
+    } else {
+        FR_CUDA_TRY(fr::launch_stream(bm->shape, bm->buf, bm->trie->dev, bm->t, logits, ld, s));
+        if (timed) FR_CUDA_TRY(cudaEventRecord(ev[1], s));
+        FR_CUDA_TRY(fr::launch_select(bm->shape, bm->buf, bm->trie->dev, bm->t, s));
+    }
     if (timed) {
         FR_CUDA_TRY(cudaEventRecord(ev[2], s));
         ++bm->n_timed;

@@ -32,516 +32,10 @@
 #include <stdint.h>
 
 #include "fr_step.cuh"
+#include "fr_topk.cuh"
 
 namespace fr {
 namespace {
-
-// ---------------------------------------------------------------------------
-// Selection and reorder.
-
-constexpr int SEL_THREADS = 1024;
-constexpr int HBITS = 12;
-constexpr int HBINS = 1 << HBITS;
-static_assert(HBINS == 4 * SEL_THREADS, "each thread owns four histogram bins");
-static_assert(FR_MAX_K <= SEL_THREADS, "one thread per beam slot");
-static_assert(HBINS * sizeof(int32_t) >= FR_MAX_K * sizeof(unsigned long long), "histogram doubles as sort scratch");
-
-struct SelectArgs {
-    StateDev cur, nxt;
-    TrieDev trie;
-    int32_t B, K, D, t;
-    const float* cand;  // candidate scores (what survivors keep)
-    const float* rank;  // what the selection ranks: cand, or the perturbed keys
-    int64_t cand_stride;
-    int32_t* parent_out;
-    int32_t* token_out;
-    int32_t* err;
-    int32_t key_cap;   // cluster select: keys each CTA's shared memory holds
-    int32_t pool_cap;  // cluster select: values the leader's pool holds
-};
-
-__device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t* out_or) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v_and = __reduce_and_sync(0xffffffffu, v_and);
-    v_or = __reduce_or_sync(0xffffffffu, v_or);
-    if (lane == 0) {
-        red[warp] = v_and;
-        red[32 + warp] = v_or;
-    }
-    __syncthreads();
-    const int nw = blockDim.x >> 5;
-    uint32_t a = 0xFFFFFFFFu, o = 0u;
-    for (int w = 0; w < nw; ++w) {
-        a &= red[w];
-        o |= red[32 + w];
-    }
-    __syncthreads();
-    *out_or = o;
-    return a;
-}
-
-// Next step's candidate offsets of request b: exclusive scan over slots of
-// the child counts of each live slot's node.  Called by all threads.
-__device__ __forceinline__ void write_cand_off(const TrieDev& trie, int t_next, const int32_t* node_row, int live,
-                                               int K, int32_t* cand_off_row) {
-    const int j = threadIdx.x;
-    int cnt = 0;
-    if (j < live) {
-        const int32_t n = node_row[j];
-        if (n >= 0) {
-            int32_t lo, hi;
-            trie_children(trie, t_next, n, lo, hi);
-            cnt = hi - lo;
-        }
-    }
-    int tot;
-    const int e = block_excl_scan(cnt, &tot);
-    if (j < K) cand_off_row[j] = e;
-    if (j == 0) cand_off_row[K] = tot;
-}
-
-// Sorts the Kp winners in sel (descending (key, ~slot), so key descending,
-// then slot ascending) and writes the request's next state: the reorder
-// gathers and the next step's candidate offsets.  All threads of the block
-// (blockDim.x >= K) call it.
-// Sorts the n (<= blockDim.x) distinct nonzero values sel[0..n) into
-// descending order.  Up to 256 values: by counting ranks.  More: a bitonic
-// network over P = max(32, next power of two >= n)
-// values held one per thread by threads 0..P-1, padded with 0 (below every
-// real value).  Compare-exchange partners closer than 32 are in the same warp
-// (shuffles); the farther ones exchange through shared memory, alternating
-// between `buf` (P values of scratch) and sel so that each such stage needs
-// one barrier, a named barrier over the P participating threads only.  All
-// threads of the block call it.
-__device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ void sort_desc_u64(unsigned long long* sel, unsigned long long* buf, int n) {
-    const int tid = threadIdx.x;
-    if (n <= 256) {
-        // few values: each one's position is the number of values above it,
-        // counted over all n (every lane of a warp reads the same value, a
-        // broadcast, two values per 16-byte load)
-        unsigned long long v = 0ull;
-        int rank = 0;
-        if (tid < n) {
-            v = sel[tid];
-            const ulonglong2* s2 = reinterpret_cast<const ulonglong2*>(sel);
-            int j = 0;
-#pragma unroll 4
-            for (; j + 1 < n; j += 2) {
-                const ulonglong2 p = s2[j >> 1];
-                rank += (p.x > v) + (p.y > v);
-            }
-            if (j < n) rank += sel[j] > v;
-        }
-        __syncthreads();
-        if (tid < n) sel[rank] = v;
-        __syncthreads();
-        return;
-    }
-    int P = 32;
-    while (P < n) P <<= 1;
-    if (tid < P) {  // whole warps: P is a multiple of 32
-        unsigned long long v = tid < n ? sel[tid] : 0ull;
-        int par = 0;
-        for (int k = 2; k <= P; k <<= 1) {
-            for (int j = k >> 1; j > 0; j >>= 1) {
-                unsigned long long o;
-                if (j >= 32) {
-                    unsigned long long* x = par ? sel : buf;
-                    x[tid] = v;
-                    bar_sync_named(1, P);
-                    o = x[tid ^ j];
-                    par ^= 1;
-                } else {
-                    o = __shfl_xor_sync(0xffffffffu, v, j);
-                }
-                const bool keep_max = ((tid & j) == 0) == ((tid & k) == 0);
-                v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
-            }
-        }
-        bar_sync_named(1, P);
-        if (tid < n) sel[tid] = v;
-    }
-    __syncthreads();
-}
-
-// Per live parent slot k of request b, read before the wait on the row kernel
-// (the previous step's selection or the reset wrote them): its candidates'
-// offset (s_off, live + 1 entries), the first level-(t+1) node of its trie
-// children (s_lo; -1 for a node outside the trie) and its KV slot (s_kv).
-// All threads of the block call it; a __syncthreads must follow before use.
-__device__ __forceinline__ void load_parents(const SelectArgs& a, int b, int live, int32_t* s_off, int32_t* s_lo,
-                                             int32_t* s_kv) {
-    const int K = a.K, t = a.t;
-    for (int i = threadIdx.x; i <= live; i += blockDim.x) s_off[i] = a.cur.cand_off[(int64_t)b * (K + 1) + i];
-    for (int k = threadIdx.x; k < live; k += blockDim.x) {
-        const int64_t ok = (int64_t)b * K + k;
-        const int32_t np = a.cur.node[ok];
-        int32_t lo = -1, hi = -1;
-        if (np >= 0 && np < a.trie.nodes[t]) trie_children(a.trie, t, np, lo, hi);
-        s_lo[k] = lo;
-        s_kv[k] = a.cur.kv[ok];
-    }
-}
-
-__device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, const int32_t* s_lo,
-                                 const int32_t* s_kv, int Kp, unsigned long long* sel, unsigned long long* scratch) {
-    const int tid = threadIdx.x;
-    const int K = a.K, D = a.D, t = a.t;
-    sort_desc_u64(sel, scratch, Kp);
-
-    // emit survivors (thread j = slot j)
-    const int j = tid;
-    int32_t child = -1;
-    if (j < K) {
-        const int64_t oj = (int64_t)b * K + j;
-        if (j < Kp) {
-            const unsigned long long v = sel[j];
-            const uint32_t key = (uint32_t)(v >> 32);
-            const int32_t slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
-            int lo = 0, hi = live - 1;  // parent: last k with s_off[k] <= slot
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
-            }
-            const int k = lo;
-            const int64_t ok = (int64_t)b * K + k;
-            int32_t tok = -1;
-            if (s_lo[k] >= 0) {
-                child = s_lo[k] + (slot - s_off[k]);
-                if (child >= 0 && child < a.trie.nodes[t + 1]) {
-                    tok = a.trie.tok_base[t] + trie_child_code(a.trie, t, child);
-                } else {
-                    child = -1;
-                }
-            }
-            if (child < 0) set_error(a.err, FR_ERR_DEVICE);
-            a.nxt.node[oj] = child;
-            a.nxt.score[oj] = (a.rank == a.cand) ? key_to_float(key) : a.cand[(int64_t)b * a.cand_stride + slot];
-            a.nxt.kv[oj] = s_kv[k];
-            a.parent_out[oj] = k;
-            a.token_out[oj] = tok;
-            for (int l = 0; l < D; ++l)
-                a.nxt.prefix[oj * D + l] = (l < t) ? a.cur.prefix[ok * D + l] : (l == t ? tok : -1);
-        } else {
-            a.nxt.node[oj] = -1;
-            a.nxt.score[oj] = -INFINITY;
-            a.nxt.kv[oj] = -1;
-            a.parent_out[oj] = -1;
-            a.token_out[oj] = -1;
-            for (int l = 0; l < D; ++l) a.nxt.prefix[oj * D + l] = -1;
-        }
-    }
-    if (tid == 0) a.nxt.live[b] = Kp;
-    if (t + 1 < D) {
-        // node ids of the survivors are in registers of threads 0..Kp-1
-        const int jj = threadIdx.x;
-        int cnt = 0;
-        if (jj < Kp && child >= 0) {
-            int32_t lo, hi;
-            trie_children(a.trie, t + 1, child, lo, hi);
-            cnt = hi - lo;
-        }
-        int tot;
-        const int e = block_excl_scan(cnt, &tot);
-        int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
-        if (jj < K) row[jj] = e;
-        if (jj == 0) row[K] = tot;
-    }
-}
-
-
-// Candidate values for the selection: val(i) = (key << 32) | low, with key an
-// order-preserving image of the candidate's score (or sampling key) and low =
-// ~slot, so that larger values come first in the step's total order (key
-// descending, slot ascending) and index order is slot order.
-// QUADS: keys 4q .. 4q+3 come from one 16-byte load, key4(q) (only then defined).  val_of(i, k)
-// is val(i) for a key k already loaded.
-struct GlobalCands {  // the request's candidates in global memory, slot i at cb[i] (cb 16-byte aligned)
-    static constexpr bool QUADS = true;
-    const float* cb;
-    __device__ __forceinline__ uint32_t key(int i) const { return float_to_key(__ldg(cb + i)); }
-    __device__ __forceinline__ uint4 key4(int q) const {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(cb) + q);
-        return make_uint4(float_to_key(x.x), float_to_key(x.y), float_to_key(x.z), float_to_key(x.w));
-    }
-    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t k) const {
-        return ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)i);
-    }
-    __device__ __forceinline__ unsigned long long val(int i) const { return val_of(i, key(i)); }
-};
-struct SmemKeys {  // a contiguous slice of them, as keys in shared memory, slot base + i at keys[i]
-    static constexpr bool QUADS = false;
-    const uint32_t* keys;
-    uint32_t base;
-    __device__ __forceinline__ uint32_t key(int i) const { return keys[i]; }
-    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t k) const {
-        return ((unsigned long long)k << 32) | (0xFFFFFFFFu - (base + (uint32_t)i));
-    }
-    __device__ __forceinline__ unsigned long long val(int i) const { return val_of(i, keys[i]); }
-};
-struct PoolVals {  // values already formed, in slot order
-    static constexpr bool QUADS = false;
-    const unsigned long long* pool;
-    __device__ __forceinline__ uint32_t key(int i) const { return (uint32_t)(pool[i] >> 32); }
-    __device__ __forceinline__ unsigned long long val_of(int i, uint32_t) const { return pool[i]; }
-    __device__ __forceinline__ unsigned long long val(int i) const { return pool[i]; }
-};
-
-// Calls f(i, key(i)) for the indices i in [0, n) this thread owns (which ones
-// depends on the access width), with eight independent loads in flight per
-// thread.  The calls' order is not index order.
-template <class Vals, class F>
-__device__ __forceinline__ void for_keys(const Vals& vals, int n, F&& f) {
-    const int tid = threadIdx.x;
-    if constexpr (Vals::QUADS) {
-        const int nq = n >> 2;
-        int q0 = tid;
-        for (; q0 + 7 * SEL_THREADS < nq; q0 += 8 * SEL_THREADS) {
-            uint4 k4[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) k4[u] = vals.key4(q0 + u * SEL_THREADS);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = (q0 + u * SEL_THREADS) * 4;
-                f(i, k4[u].x);
-                f(i + 1, k4[u].y);
-                f(i + 2, k4[u].z);
-                f(i + 3, k4[u].w);
-            }
-        }
-        for (int q = q0; q < nq; q += SEL_THREADS) {
-            const uint4 k4 = vals.key4(q);
-            f(4 * q, k4.x);
-            f(4 * q + 1, k4.y);
-            f(4 * q + 2, k4.z);
-            f(4 * q + 3, k4.w);
-        }
-        const int i = 4 * nq + tid;  // the last n mod 4
-        if (i < n) f(i, vals.key(i));
-    } else {
-        int i0 = tid;
-        for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-            uint32_t k8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) k8[u] = vals.key(i0 + u * SEL_THREADS);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) f(i0 + u * SEL_THREADS, k8[u]);
-        }
-        for (int i = i0; i < n; i += SEL_THREADS) f(i, vals.key(i));
-    }
-}
-
-// Exact top-Kp (Kp <= n, Kp <= FR_MAX_K) of the n values under the total
-// order: the Kp winners' values go to out[0..Kp); the return value is how
-// many were written (Kp unless something is inconsistent).  The Kp-th key T
-// is found by radix selection on the keys (12-bit digits after skipping the
-// bits every key shares); the winners are every key > T and the lowest-index
-// keys == T.  The search stops early once the bin holding the Kp-th key holds
-// exactly the keys still needed: T is then that bin's lowest value, and the
-// winners are the keys >= T.  ORDERED: they are written in index (slot) order -- each warp
-// owns a contiguous block of indices and counts its keys above and at T
-// (ballots), one scan over the warps gives each warp its output offset, and a
-// second sweep writes.  Otherwise in any order, in one sweep (atomic
-// positions; when not all the keys equal to T win, their lowest indices are
-// found by ranking them, or, past SEL_THREADS of them, by block scans in index
-// order).  All threads of the block call it; scratch:
-// hist [HBINS], red [64], s_misc [8].
-template <bool ORDERED, class Vals>
-__device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* out, int32_t* hist, uint32_t* red,
-                          int32_t* s_misc) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (Kp <= 0 || n <= 0) return 0;
-    uint32_t T = 0u;
-    int eq_needed = n;  // Kp == n: every value wins (all keys are >= 0)
-    int count_eq = n;   // keys equal to T (an upper bound when every value wins)
-    if (Kp < n) {
-        uint32_t va = 0xFFFFFFFFu, vo = 0u;
-        for_keys(vals, n, [&](int, uint32_t k) {
-            va &= k;
-            vo |= k;
-        });
-        uint32_t VO;
-        const uint32_t VA = block_and_or(va, vo, red, &VO);
-        const uint32_t diff = VA ^ VO;
-        if (diff == 0u) {
-            T = VA;
-            eq_needed = Kp;
-            count_eq = n;
-        } else {
-            int lo = 32 - __clz(diff);  // bits >= lo are the same in every key
-            uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
-            int krem = Kp;
-            while (lo > 0) {
-                const int width = min(HBITS, lo);
-                const int shift = lo - width;
-                const uint32_t dmask = (1u << width) - 1u;
-                for (int i = tid; i < HBINS; i += SEL_THREADS) hist[i] = 0;
-                __syncthreads();
-                const uint64_t want = (uint64_t)prefix >> lo;
-                for_keys(vals, n, [&](int, uint32_t k) {
-                    if (((uint64_t)k >> lo) == want) atomicAdd(&hist[(k >> shift) & dmask], 1);
-                });
-                __syncthreads();
-                int h4[4], tsum = 0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    h4[q] = hist[tid * 4 + q];
-                    tsum += h4[q];
-                }
-                int tot;
-                const int excl = block_excl_scan(tsum, &tot);
-                int cum = tot - excl - tsum;  // keys in the bins above this thread's
-#pragma unroll
-                for (int q = 3; q >= 0; --q) {
-                    if (cum < krem && cum + h4[q] >= krem) {
-                        s_misc[0] = tid * 4 + q;
-                        s_misc[1] = cum;
-                        s_misc[2] = h4[q];
-                    }
-                    cum += h4[q];
-                }
-                __syncthreads();
-                krem -= s_misc[1];
-                count_eq = s_misc[2];
-                prefix |= (uint32_t)s_misc[0] << shift;
-                lo = shift;
-                __syncthreads();
-                // Every key of the threshold bin wins: T = prefix (its lower
-                // bits zero) already splits the keys, with keys >= T winning.
-                if (count_eq == krem) break;
-            }
-            T = prefix;
-            eq_needed = krem;
-        }
-    }
-    if constexpr (!ORDERED) {
-        if (tid == 0) {
-            s_misc[3] = 0;
-            s_misc[4] = 0;
-        }
-        __syncthreads();
-        if (eq_needed >= count_eq) {  // every key >= T wins
-            for_keys(vals, n, [&](int i, uint32_t k) {
-                if (k >= T) {
-                    const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < Kp) out[p] = vals.val_of(i, k);
-                }
-            });
-        } else if (count_eq <= SEL_THREADS) {
-            // Few keys equal T (ties of equal scores): every key > T wins;
-            // the indices of the keys == T go to the histogram's space, and
-            // those with fewer than eq_needed lower indices among them win.
-            int32_t* eq_idx = hist;
-            for_keys(vals, n, [&](int i, uint32_t k) {
-                if (k > T) {
-                    const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < Kp) out[p] = vals.val_of(i, k);
-                } else if (k == T) {
-                    const int q = atomicAdd(&s_misc[4], 1);
-                    if (q < SEL_THREADS) eq_idx[q] = i;
-                }
-            });
-            __syncthreads();
-            const int ne = min(s_misc[4], SEL_THREADS);
-            if (tid < ne) {
-                const int mine = eq_idx[tid];
-                int below = 0;
-                for (int j = 0; j < ne; ++j) below += eq_idx[j] < mine;
-                if (below < eq_needed) {
-                    const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < Kp) out[p] = vals.val_of(mine, T);
-                }
-            }
-        } else {  // many keys equal T straddle the boundary: take them in index order
-            int run_eq = 0;
-            for (int base = 0; base < n; base += SEL_THREADS) {
-                const int i = base + tid;
-                const unsigned long long v = i < n ? vals.val(i) : 0ull;
-                const uint32_t k = (uint32_t)(v >> 32);
-                const bool gt = i < n && k > T;
-                const bool eq = i < n && k == T;
-                int tot;
-                const int r = block_excl_scan(eq ? 1 : 0, &tot);
-                if (gt || (eq && run_eq + r < eq_needed)) {
-                    const int p = atomicAdd(&s_misc[3], 1);
-                    if (p < Kp) out[p] = v;
-                }
-                run_eq += tot;
-            }
-        }
-        __syncthreads();
-        return s_misc[3];
-    }
-    // collect in index order
-    constexpr int NW = SEL_THREADS / 32;
-    const int per = (((n + NW - 1) / NW) + 31) & ~31;
-    const int beg = min(n, warp * per), end = min(n, beg + per);
-    constexpr int CB = 8;  // 32-wide rows per batch: CB independent loads in flight per lane
-    int cgt = 0, ceq = 0;
-    for (int j = beg; j < end; j += 32 * CB) {
-        uint32_t k8[CB];
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const int i = j + u * 32 + lane;
-            k8[u] = i < end ? vals.key(i) : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const bool in = j + u * 32 + lane < end;
-            cgt += __popc(__ballot_sync(0xffffffffu, in && k8[u] > T));
-            ceq += __popc(__ballot_sync(0xffffffffu, in && k8[u] == T));
-        }
-    }
-    if (lane == 0) {
-        red[warp] = (uint32_t)cgt;
-        red[NW + warp] = (uint32_t)ceq;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int g = lane < NW ? (int)red[lane] : 0, e = lane < NW ? (int)red[NW + lane] : 0;
-        const int gi = warp_incl_scan(g), ei = warp_incl_scan(e);
-        if (lane < NW) {
-            red[lane] = (uint32_t)(gi - g);
-            red[NW + lane] = (uint32_t)(ei - e);
-        }
-        if (lane == 31) {
-            s_misc[6] = gi;
-            s_misc[7] = ei;
-        }
-    }
-    __syncthreads();
-    int gbase = (int)red[warp], ebase = (int)red[NW + warp];
-    const int total = s_misc[6] + min(s_misc[7], eq_needed);
-    const unsigned lt = (1u << lane) - 1u;
-    for (int j = beg; j < end; j += 32 * CB) {
-        unsigned long long v8[CB];
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const int i = j + u * 32 + lane;
-            v8[u] = i < end ? vals.val(i) : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const bool in = j + u * 32 + lane < end;
-            const uint32_t k = (uint32_t)(v8[u] >> 32);
-            const bool g = in && k > T, e = in && k == T;
-            const unsigned bg = __ballot_sync(0xffffffffu, g), be = __ballot_sync(0xffffffffu, e);
-            const int gb = gbase + __popc(bg & lt), eb = ebase + __popc(be & lt);
-            int pos = -1;
-            if (g) pos = gb + min(eb, eq_needed);
-            else if (e && eb < eq_needed) pos = gb + eb;
-            if (pos >= 0 && pos < Kp) out[pos] = v8[u];
-            gbase += __popc(bg);
-            ebase += __popc(be);
-        }
-    }
-    __syncthreads();
-    return total;
-}
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     __shared__ int32_t s_off[FR_MAX_K + 1];

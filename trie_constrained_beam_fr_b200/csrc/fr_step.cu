@@ -41,6 +41,7 @@
 #include <stdint.h>
 
 #include "fr_step.cuh"
+#include "fr_topk.cuh"
 
 namespace fr {
 namespace {
@@ -933,6 +934,158 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Step 0, fused.  At the first step every request has one live beam, the
+// root, so the step streams only B rows and its selection ranks only the
+// root's children.  Run as the two general kernels, the streaming kernel's
+// pipeline never fills and the selection pays its own launch; here one kernel
+// does the whole step: the root row of request b is cut into `parts` equal
+// pieces, one CTA each (16-byte vectors, a batch of ROOT_VPL per thread in
+// flight, each batch's maximum first and then its exponent sum against the
+// running maximum); each CTA leaves its (max, scaled sum) and the last CTA of
+// the request to arrive (atomic counter, no waiting) combines them in piece
+// order, writes the root's children's scores as keys in shared memory and
+// runs the selection routine of k_select on them: top-K under the total
+// order, sort, reorder gathers and next candidate offsets.  Used at
+// temperature 0 over the full vocabulary when the root has at most
+// ROOT_MAX_CANDS children.
+
+constexpr int ROOT_THREADS = SEL_THREADS;  // the selection routine's block size
+constexpr int ROOT_MAX_CANDS = 8192;       // root children held as keys (32 KB of shared memory)
+constexpr int ROOT_MAX_PARTS = 64;         // pieces per root row
+constexpr int ROOT_VPL = 4;                // 16-byte vectors per thread per batch
+
+template <bool BF16>
+__global__ void __launch_bounds__(ROOT_THREADS, 1)
+    k_root_step(const StreamArgs a, const SelectArgs sl, int32_t parts, float2* __restrict__ rpart) {
+    constexpr int ELT = BF16 ? 2 : 4;
+    constexpr int64_t VE = 16 / ELT;
+    extern __shared__ __align__(16) uint32_t keys[];  // [ROOT_MAX_CANDS]
+    __shared__ __align__(16) int32_t hist[HBINS];    // also the sort's scratch
+    __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
+    __shared__ int32_t s_off[2];
+    __shared__ int32_t s_lo[1];
+    __shared__ int32_t s_kv[1];
+    __shared__ uint32_t red[64];
+    __shared__ int32_t s_misc[8];
+    __shared__ float2 wpart[ROOT_THREADS / 32];
+    __shared__ float s_lse;
+    __shared__ int32_t s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int p = blockIdx.x, b = blockIdx.y;
+    const int K = a.K;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int live = min(max(a.live[b], 0), 1);  // at step 0: the root or nothing
+    if (live == 0) {
+        if (p != 0) return;
+        // no beam at all: the request's next state is all dead
+        if (tid == 0) s_off[0] = s_off[1] = 0;
+        __syncthreads();
+        select_sort_emit(sl, b, 0, s_off, s_lo, s_kv, 0, sel, reinterpret_cast<unsigned long long*>(hist));
+        return;
+    }
+    const int64_t bk = (int64_t)b * K;  // the root is slot 0
+    const char* row = a.logits + bk * a.ld * ELT;
+    const char* win = row + a.col0 * ELT;
+    const int64_t W = a.W;
+    const int64_t per = ((W + parts - 1) / parts + VE - 1) / VE * VE;
+    const int64_t c0 = min(W, (int64_t)p * per), c1 = min(W, c0 + per);
+    const uint32_t mis = (uint32_t)(reinterpret_cast<uint64_t>(win) + (uint64_t)(c0 * ELT)) & 15u;
+    const int64_t a0 = min(c0 + (int64_t)((16u - mis) & 15u) / ELT, c1);
+    const int64_t nvec = (c1 - a0) / VE;
+    const int64_t a1 = a0 + nvec * VE;
+    const uint4* vec = reinterpret_cast<const uint4*>(win + a0 * ELT);
+    const uint32_t ninf = BF16 ? 0xFF80FF80u : 0xFF800000u;
+    const uint4 ninf4 = make_uint4(ninf, ninf, ninf, ninf);
+
+    float m = -INFINITY;
+    f32x2 s2 = 0ull;
+    for (int64_t v0 = 0; v0 < nvec; v0 += (int64_t)ROOT_THREADS * ROOT_VPL) {
+        uint4 q[ROOT_VPL];
+#pragma unroll
+        for (int j = 0; j < ROOT_VPL; ++j) {
+            const int64_t i = v0 + (int64_t)j * ROOT_THREADS + tid;
+            q[j] = i < nvec ? __ldg(vec + i) : ninf4;
+        }
+        const float mn = fmax_nan(m, lane_max<BF16>(q));
+        if (m != -INFINITY && mn != m) {
+            const float sc = ex2_approx((m - mn) * L2E);  // NaN when mn is NaN
+            s2 = mul2(s2, pack2(sc, sc));
+        }
+        m = mn;
+        if (m != -INFINITY) s2 = add2(s2, lane_expsum<BF16>(q, m));
+    }
+    for (int64_t i = c0 + tid; i < a0; i += ROOT_THREADS) lane_add(m, s2, load_elem(win, i, ELT));
+    for (int64_t i = a1 + tid; i < c1; i += ROOT_THREADS) lane_add(m, s2, load_elem(win, i, ELT));
+    float lo2, hi2;
+    unpack2(s2, lo2, hi2);
+    float s = lo2 + hi2;
+    warp_combine(m, s);
+    if (lane == 0) wpart[warp] = make_float2(m, s);
+    __syncthreads();
+    if (warp == 0) {
+        float pm = wpart[lane].x, ps = wpart[lane].y;
+        warp_combine(pm, ps);
+        if (lane == 0) {
+            rpart[(int64_t)b * parts + p] = make_float2(pm, ps);
+            __threadfence();
+            s_last = atomicAdd(&a.row_cnt[bk], 1) == parts - 1;
+        }
+    }
+    __syncthreads();
+    if (!s_last) return;
+    // the last piece of the row has arrived: combine the pieces in order
+    __threadfence();
+    if (warp == 0) {
+        float M = -INFINITY, S = 0.f;
+        for (int base = 0; base < parts; base += 32) {
+            const int g = base + lane;
+            float pm = -INFINITY, ps = 0.f;
+            if (g < parts) {
+                const float2 q = __ldcg(&rpart[(int64_t)b * parts + g]);
+                pm = q.x;
+                ps = q.y;
+            }
+            warp_combine(pm, ps);
+            combine(M, S, pm, ps);
+        }
+        if (lane == 0) {
+            s_lse = M + logf(S);
+            a.row_cnt[bk] = 0;
+            if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
+        }
+    }
+    // the root's children: candidate slot i is child i (code order)
+    const int32_t n0 = a.node[bk];
+    int32_t clo = -1, chi = -1;
+    if (n0 >= 0 && n0 < a.trie.nodes[0]) trie_children(a.trie, 0, n0, clo, chi);
+    int32_t nch = chi - clo;
+    if (clo < 0 || nch < 0 || nch > ROOT_MAX_CANDS || a.cand_off[(int64_t)b * (K + 1)] != 0) {
+        if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
+        nch = 0;
+    }
+    __syncthreads();
+    const float lse = s_lse;
+    const float sc = a.score[bk];
+    const int32_t* codes = a.trie.code[1] + clo;
+    const bool dense = a.trie.dense_c[0] != 0;
+    const int32_t tb = a.trie.tok_base[0];
+    for (int32_t i = tid; i < nch; i += ROOT_THREADS)
+        keys[i] = float_to_key(sc + (load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT) - lse));
+    if (tid == 0) {
+        s_off[0] = 0;
+        s_off[1] = nch;
+        s_lo[0] = clo;
+        s_kv[0] = sl.cur.kv[bk];
+    }
+    __syncthreads();
+    const int Kp = min(K, nch);
+    const int got = block_topk<false>(SmemKeys{keys, 0u}, nch, Kp, sel, hist, red, s_misc);
+    if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
+    select_sort_emit(sl, b, 1, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+}
+
 }  // namespace
 
 size_t stream_smem_bytes(int32_t B, bool bf16) {
@@ -994,6 +1147,69 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     StepLaunch L(dim3((unsigned)sh.grid), STREAM_THREADS, stream_smem_bytes(sh.B, sh.dtype == FR_BF16), s);
     return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_stream<true>, a)
                                : cudaLaunchKernelEx(&L.cfg, k_stream<false>, a);
+}
+
+bool root_step_fused(const StepShape& sh, const TrieDev& trie) {
+    const int64_t row_bytes = (int64_t)sh.V * (sh.dtype == FR_BF16 ? 2 : 4);
+    return sh.norm == FR_NORM_FULL && !(sh.inv_temp > 0.f) && !sh.starve && trie.nodes[1] <= ROOT_MAX_CANDS &&
+           row_bytes > SHORT_ROW_BYTES;
+}
+
+cudaError_t root_step_setup() {
+    cudaError_t e = cudaFuncSetAttribute(k_root_step<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(ROOT_MAX_CANDS * sizeof(uint32_t)));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_root_step<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(ROOT_MAX_CANDS * sizeof(uint32_t)));
+}
+
+int32_t root_step_max_parts() { return ROOT_MAX_PARTS; }
+
+cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, const void* logits,
+                             int64_t ld, cudaStream_t s) {
+    const StateDev& cur = buf.st[0];
+    StreamArgs a{};
+    a.logits = static_cast<const char*>(logits);
+    a.ld = ld;
+    a.V = sh.V;
+    a.B = sh.B;
+    a.K = sh.K;
+    a.t = 0;
+    a.elt = sh.dtype == FR_BF16 ? 2 : 4;
+    a.col0 = 0;
+    a.W = sh.V;
+    a.live = cur.live;
+    a.node = cur.node;
+    a.score = cur.score;
+    a.cand_off = cur.cand_off;
+    a.trie = trie;
+    a.row_cnt = buf.row_cnt;
+    a.err = buf.err;
+    a.wait_ns = FR_WAIT_LIMIT_NS;
+    SelectArgs sl{};
+    sl.cur = cur;
+    sl.nxt = buf.st[1];
+    sl.trie = trie;
+    sl.B = sh.B;
+    sl.K = sh.K;
+    sl.D = sh.D;
+    sl.t = 0;
+    sl.cand = buf.cand;
+    sl.rank = buf.cand;  // temperature 0: survivors' scores are their keys
+    sl.cand_stride = buf.cand_stride;
+    sl.parent_out = buf.parent;
+    sl.token_out = buf.token;
+    sl.err = buf.err;
+    // one CTA per SM in all (measured on B200 against two per SM and against
+    // more vectors per batch), each piece at least 8,192 elements
+    int32_t parts = (int32_t)((int64_t)sh.grid / sh.B);
+    const int32_t by_len = (int32_t)((sh.V + 8191) / 8192);
+    parts = parts < by_len ? parts : by_len;
+    parts = parts < ROOT_MAX_PARTS ? parts : ROOT_MAX_PARTS;
+    parts = parts > 1 ? parts : 1;
+    StepLaunch L(dim3((unsigned)parts, (unsigned)sh.B), ROOT_THREADS, ROOT_MAX_CANDS * sizeof(uint32_t), s);
+    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_root_step<true>, a, sl, parts, buf.root_partial)
+                               : cudaLaunchKernelEx(&L.cfg, k_root_step<false>, a, sl, parts, buf.root_partial);
 }
 
 cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
