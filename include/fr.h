@@ -273,7 +273,7 @@ fr_status fr_beam_set_sampling(fr_beam* beam, float temperature, uint64_t seed, 
  * (stream_ms: the fused log-sum-exp / candidate kernel, select_ms: the top-K
  * and reorder kernel) in step order, stores the count in *n, and clears.
  * The first step runs as one kernel when every request starts from its root
- * (temperature 0, full vocabulary, rows longer than 16 KB, at most 8,192 root
+ * (temperature 0, full vocabulary or SID range, at most 8,192 root
  * children): its whole time is in stream_ms and select_ms is the gap between
  * two back-to-back events. */
 fr_status fr_beam_set_timing(fr_beam* beam, int32_t enable);

@@ -79,7 +79,8 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
         delete bm;
         return FR_ERR_CUDA;
     }
-    if (fr::stream_kernel_setup() != cudaSuccess || fr::root_step_setup() != cudaSuccess) {
+    if (fr::stream_kernel_setup() != cudaSuccess || fr::root_step_setup() != cudaSuccess ||
+        fr::select_kernel_setup() != cudaSuccess) {
         (void)cudaGetLastError();
         delete bm;
         return FR_ERR_CUDA;

@@ -37,7 +37,15 @@
 namespace fr {
 namespace {
 
+// STAGED: the request's candidates (at most key_cap of them) are read once
+// into shared memory as keys and every pass of the selection reads them from
+// there; otherwise every pass reads them from global memory (L2).  Two
+// instantiations so that the global-memory version keeps its own code.
+constexpr int64_t SEL_STAGE_CAP = 16384;  // keys (64 KB of shared memory)
+
+template <bool STAGED>
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
+    extern __shared__ __align__(16) uint32_t skeys[];  // STAGED: [key_cap] the candidates as keys
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ int32_t s_lo[FR_MAX_K];
     __shared__ int32_t s_kv[FR_MAX_K];
@@ -55,12 +63,26 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     griddep_launch_dependents();
     __syncthreads();
     int n = s_off[live];
-    if (n < 0 || (int64_t)n > a.cand_stride) {
+    if (n < 0 || (int64_t)n > a.cand_stride || (STAGED && n > a.key_cap)) {
         if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
         n = 0;
     }
     const int Kp = min(K, n);
-    const int got = block_topk<false>(GlobalCands{a.rank + (int64_t)b * a.cand_stride}, n, Kp, sel, hist, red, s_misc);
+    int got;
+    if constexpr (STAGED) {
+        const float* cb = a.rank + (int64_t)b * a.cand_stride;  // 16-byte aligned
+        const int nq = n >> 2;
+        for (int q = tid; q < nq; q += SEL_THREADS) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(cb) + q);
+            reinterpret_cast<uint4*>(skeys)[q] =
+                make_uint4(float_to_key(x.x), float_to_key(x.y), float_to_key(x.z), float_to_key(x.w));
+        }
+        if (4 * nq + tid < n) skeys[4 * nq + tid] = float_to_key(__ldg(cb + 4 * nq + tid));
+        __syncthreads();
+        got = block_topk<false>(SmemKeys{skeys, 0u}, n, Kp, sel, hist, red, s_misc);
+    } else {
+        got = block_topk<false>(GlobalCands{a.rank + (int64_t)b * a.cand_stride}, n, Kp, sel, hist, red, s_misc);
+    }
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
     select_sort_emit(a, b, live, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
 }
@@ -274,13 +296,24 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
     a.err = buf.err;
     const int cs = sh.sel_cluster[t];
     if (cs <= 0) {
+        const int64_t bound = sh.sel_bound[t];
+        if (bound <= SEL_STAGE_CAP) {
+            a.key_cap = (int32_t)((bound + 3) & ~(int64_t)3);
+            StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, sizeof(uint32_t) * (size_t)a.key_cap, s);
+            return cudaLaunchKernelEx(&L.cfg, k_select<true>, a);
+        }
         StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, 0, s);
-        return cudaLaunchKernelEx(&L.cfg, k_select, a);
+        return cudaLaunchKernelEx(&L.cfg, k_select<false>, a);
     }
     a.key_cap = (int32_t)((sh.sel_bound[t] + cs - 1) / cs);
     a.pool_cap = cs * (sh.K < a.key_cap ? sh.K : a.key_cap);
     StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, csel_smem_bytes(a.key_cap, cs, sh.K), s, (unsigned)cs);
     return cudaLaunchKernelEx(&L.cfg, k_select_cluster, a);
+}
+
+cudaError_t select_kernel_setup() {
+    return cudaFuncSetAttribute(k_select<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(SEL_STAGE_CAP * sizeof(uint32_t)));
 }
 
 int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {

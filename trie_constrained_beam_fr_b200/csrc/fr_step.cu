@@ -947,8 +947,8 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
 // order, writes the root's children's scores as keys in shared memory and
 // runs the selection routine of k_select on them: top-K under the total
 // order, sort, reorder gathers and next candidate offsets.  Used at
-// temperature 0 over the full vocabulary when the root has at most
-// ROOT_MAX_CANDS children.
+// temperature 0 over the full vocabulary or the SID token range when the root
+// has at most ROOT_MAX_CANDS children.
 
 constexpr int ROOT_THREADS = SEL_THREADS;  // the selection routine's block size
 constexpr int ROOT_MAX_CANDS = 8192;       // root children held as keys (32 KB of shared memory)
@@ -1150,9 +1150,8 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
 }
 
 bool root_step_fused(const StepShape& sh, const TrieDev& trie) {
-    const int64_t row_bytes = (int64_t)sh.V * (sh.dtype == FR_BF16 ? 2 : 4);
-    return sh.norm == FR_NORM_FULL && !(sh.inv_temp > 0.f) && !sh.starve && trie.nodes[1] <= ROOT_MAX_CANDS &&
-           row_bytes > SHORT_ROW_BYTES;
+    return (sh.norm == FR_NORM_FULL || sh.norm == FR_NORM_SID_RANGE) && !(sh.inv_temp > 0.f) && !sh.starve &&
+           trie.nodes[1] <= ROOT_MAX_CANDS;
 }
 
 cudaError_t root_step_setup() {
@@ -1176,8 +1175,8 @@ cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const 
     a.K = sh.K;
     a.t = 0;
     a.elt = sh.dtype == FR_BF16 ? 2 : 4;
-    a.col0 = 0;
-    a.W = sh.V;
+    a.col0 = sh.norm == FR_NORM_SID_RANGE ? trie.tok_base[0] : 0;  // the window each row normalises over
+    a.W = sh.norm == FR_NORM_SID_RANGE ? sh.sid_span : sh.V;
     a.live = cur.live;
     a.node = cur.node;
     a.score = cur.score;
@@ -1203,7 +1202,7 @@ cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const 
     // one CTA per SM in all (measured on B200 against two per SM and against
     // more vectors per batch), each piece at least 8,192 elements
     int32_t parts = (int32_t)((int64_t)sh.grid / sh.B);
-    const int32_t by_len = (int32_t)((sh.V + 8191) / 8192);
+    const int32_t by_len = (int32_t)((a.W + 8191) / 8192);
     parts = parts < by_len ? parts : by_len;
     parts = parts < ROOT_MAX_PARTS ? parts : ROOT_MAX_PARTS;
     parts = parts > 1 ? parts : 1;

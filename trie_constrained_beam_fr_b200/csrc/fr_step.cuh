@@ -73,6 +73,7 @@ inline int small_grid(int64_t n) {
 // Cluster size of the selection for a step whose requests have at most
 // `bound` candidates (0 = the single-CTA kernel).
 int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms);
+cudaError_t select_kernel_setup();  // raises the one-CTA selection's shared-memory limit
 
 // Streaming kernel: dynamic shared memory it needs for B requests (bf16 or
 // fp32 rows: the ring differs).
@@ -83,8 +84,8 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
                           const void* logits, int64_t ld, cudaStream_t s);
 // Step 0 as one kernel (root rows + selection) instead of launch_stream +
 // launch_select: used when root_step_fused() holds (temperature 0, full
-// vocabulary, rows longer than the short-row threshold, at most 8,192 root
-// children, no wait test setting).  root_step_setup raises its shared-memory
+// vocabulary or SID range, at most 8,192 root children, no wait test
+// setting).  root_step_setup raises its shared-memory
 // limit (once per device).
 bool root_step_fused(const StepShape& sh, const TrieDev& trie);
 cudaError_t root_step_setup();
