@@ -33,7 +33,7 @@ METRIC = "constrained beam candidates/sec (B·K·steps/s) and logits HBM GB/s vs
 UNIT = "candidates/s"
 # the streaming kernel's translation unit: its source and the headers it includes
 STREAM_KERNEL_SRC = [os.path.join(ROOT, "trie_constrained_beam_fr_b200", "csrc", f)
-                     for f in ("fr_step.cu", "fr_step.cuh", "fr_internal.cuh")]
+                     for f in ("fr_step.cu", "fr_step.cuh", "fr_internal.cuh", "fr_topk.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -116,9 +116,10 @@ def kernel_source_hash() -> str:
     return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
-def recorded_traffic(config: str):
-    """Per-launch DRAM bytes of the streaming kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
+def recorded_traffic(config: str, live_rows_per_launch: float):
+    """Per-launch DRAM bytes (read + written) of the streaming kernel: the
+    committed ncu capture's bytes per live row, times the launch's average
+    live rows, if the capture was taken on the current kernel source."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
@@ -126,7 +127,7 @@ def recorded_traffic(config: str):
     e = d.get(config)
     if not e or e.get("kernel_sha") != kernel_source_hash():
         return None
-    return e.get("bytes_per_launch")
+    return e["bytes_per_live_row"] * live_rows_per_launch
 
 
 class ClockSampler:
@@ -589,6 +590,8 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
         fr.fr_beam_set_sampling(beam, args.temperature, 0x5EED, b_offset)
     # columns each live row's log-sum-exp streams (none over the candidate slice)
     row_cols = {"full": V, "sid_range": sum(w.codebook_sizes), "candidates": 0}[args.norm]
+    # the first step runs as one kernel (root rows + selection) under these settings
+    fused0 = fr.fr_beam_fused_first_step(beam)
 
     # one untimed decode produces every step's logits (prefix-dependent)
     bufs = [torch.empty((B, K, V), dtype=tdt, device=dev) for _ in range(D)]
@@ -652,29 +655,38 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
     cands_per_decode = B * K * D
     value = job_throughput(world, cands_per_decode, args.steps, elapsed_ms)
 
-    # roofline of the dominant kernel: the streaming log-sum-exp / candidate kernel
+    # roofline of the dominant kernel: the streaming log-sum-exp / candidate
+    # kernel, over its own launches (not the fused first step's)
     peak, peak_kind = measured_peaks()
     n_launch = len(stream_ms)
     per_step_bytes = [r * row_cols * elt for r in rows]
-    alg_bytes = sum(per_step_bytes[i % D] for i in range(n_launch))
-    stream_total_ms = float(np.sum(stream_ms))
-    achieved = alg_bytes / (stream_total_ms / 1e3) / 1e9
     row_kernel = ("k_slice_candidates" if not row_cols else
                   "k_rows_short" if row_cols * elt <= 16384 else "k_stream")
+    idx = [i for i in range(n_launch) if not (fused0 and i % D == 0)]
+    alg_bytes = sum(per_step_bytes[i % D] for i in idx)
+    stream_total_ms = float(sum(stream_ms[i] for i in idx))
+    achieved = alg_bytes / (stream_total_ms / 1e3) / 1e9 if stream_total_ms > 0 else 0.0
+    live_rows_per_launch = sum(rows[i % D] for i in idx) / max(1, len(idx))
     # the committed counters are for k_stream over the full vocabulary
-    traffic = recorded_traffic(w.name) if (args.norm == "full" and row_kernel == "k_stream") else None
+    traffic = (recorded_traffic(w.name, live_rows_per_launch)
+               if (args.norm == "full" and row_kernel == "k_stream") else None)
     roofline = {"bound": "hbm" if row_cols else "latency", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
                 "kernel": row_kernel, "timing": "per-kernel CUDA events, second timed pass of the same decodes",
-                "alg_bytes_per_launch": alg_bytes / max(1, n_launch),
-                "ms_per_launch": stream_total_ms / max(1, n_launch),
+                "launches": "steps %s of each decode" % ("1.." + str(D - 1) if fused0 else "0.." + str(D - 1)),
+                "alg_bytes_per_launch": alg_bytes / max(1, len(idx)),
+                "ms_per_launch": stream_total_ms / max(1, len(idx)),
                 "frac_of_8tbs": achieved / 8000.0}
     per_step = []
     for t in range(D):
         sm = [stream_ms[i] for i in range(t, n_launch, D)]
         se = [select_ms[i] for i in range(t, n_launch, D)]
-        per_step.append({"t": t, "live_rows": rows[t], "stream_us": 1e3 * float(np.mean(sm)),
-                         "select_us": 1e3 * float(np.mean(se)),
+        one = fused0 and t == 0
+        per_step.append({"t": t, "live_rows": rows[t],
+                         "kernels": ("k_root_step (rows and selection in one kernel)" if one else
+                                     "%s + selection" % row_kernel),
+                         "stream_us": 1e3 * float(np.mean(sm)),
+                         "select_us": None if one else 1e3 * float(np.mean(se)),
                          "stream_gbs": per_step_bytes[t] / (float(np.mean(sm)) / 1e3) / 1e9 if sm else 0.0})
     hbm_gbs_decode = bytes_per_decode / (ms_per_decode / 1e3) / 1e9
 
@@ -729,7 +741,7 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
             "hbm_gbs": hbm_gbs_decode, "hbm_frac_of_8tbs": hbm_gbs_decode / 8000.0,
             "ms_per_step_with_kernel_events": evented_ms / args.steps, "roofline": roofline,
             "per_step": per_step, "trie_build_ms": trie_ms, "clocks": clocks.summary(), "e2e": e2e,
-            "sids_np": sids_np}
+            "gpu_launches": args.steps * (2 * D + 2 - (1 if fused0 else 0)), "sids_np": sids_np}
 
 
 # The catalog-scale workloads recorded beside the serving headline.
@@ -781,7 +793,6 @@ def main():
             r = measure_logits_workload(wo, args, dev, world, bo, barrier, slowest, with_e2e=False)
             r.pop("sids_np")
             r.pop("e2e")
-            r["gpu_launches"] = args.steps * (2 * wo.depth + 2)
             others[name] = r
 
     cpu = None
@@ -798,7 +809,7 @@ def main():
             "hbm_gbs": head["hbm_gbs"], "hbm_frac_of_8tbs": head["hbm_frac_of_8tbs"],
             "ms_per_step_with_kernel_events": head["ms_per_step_with_kernel_events"],
             "roofline": head["roofline"], "per_step": head["per_step"], "trie_build_ms": head["trie_build_ms"],
-            "gpu_launches": args.steps * (2 * w.depth + 2),
+            "gpu_launches": head["gpu_launches"],
             "clocks": head["clocks"], "e2e": head["e2e"], "cpu_baseline": cpu,
         }
         if others:

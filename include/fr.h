@@ -170,6 +170,14 @@ fr_status fr_beam_outputs(const fr_beam* beam, const int32_t** parent, const int
 /* Steps done so far (0..depth). */
 int32_t fr_beam_steps_done(const fr_beam* beam);
 
+/* 1 when the beam's first step runs as one kernel (the root rows and the
+ * selection together: temperature 0, at most 8,192 root children, no wait
+ * test setting), 0 when it runs as the row
+ * kernel and the selection kernel like every later step, -1 for NULL.  Reflects
+ * the current settings (fr_beam_set_normalization, fr_beam_set_sampling,
+ * fr_beam_set_wait_test). */
+int32_t fr_beam_fused_first_step(const fr_beam* beam);
+
 /* After `depth` steps (else FR_ERR_STATE): writes the ranked beams (async).
  *   sids_dev    device int32 [B, K, depth] codes (-1 for dead beams)
  *   scores_dev  device float [B, K] (-inf dead)
@@ -273,9 +281,9 @@ fr_status fr_beam_set_sampling(fr_beam* beam, float temperature, uint64_t seed, 
  * (stream_ms: the fused log-sum-exp / candidate kernel, select_ms: the top-K
  * and reorder kernel) in step order, stores the count in *n, and clears.
  * The first step runs as one kernel when every request starts from its root
- * (temperature 0, full vocabulary or SID range, at most 8,192 root
- * children): its whole time is in stream_ms and select_ms is the gap between
- * two back-to-back events. */
+ * (temperature 0, at most 8,192 root children; see fr_beam_fused_first_step):
+ * its whole time is in stream_ms and select_ms is the gap between two
+ * back-to-back events. */
 fr_status fr_beam_set_timing(fr_beam* beam, int32_t enable);
 fr_status fr_beam_read_timing(fr_beam* beam, float* stream_ms, float* select_ms, int32_t max_steps,
                               int32_t* n);

@@ -60,6 +60,7 @@ def test_host_side_argument_errors_need_no_gpu():
     assert L.fr_beam_init(None, 1, 8, 64, 0, None, ctypes.byref(out)) == fr.FR_ERR_INVALID_ARG
     assert L.fr_beam_step(None, None, 64, None) == fr.FR_ERR_INVALID_ARG
     assert L.fr_beam_steps_done(None) == -1
+    assert L.fr_beam_fused_first_step(None) == -1
     G = fr.libfr_gen()
     assert G.fr_gen_hash_logits(0, 0, 0, 8, 64, 64, 0, None, 0, 0, None, None, None) == fr.FR_ERR_INVALID_ARG
 

@@ -242,6 +242,11 @@ extern "C" fr_status fr_beam_outputs(const fr_beam* bm, const int32_t** parent, 
 
 extern "C" int32_t fr_beam_steps_done(const fr_beam* bm) { return bm ? bm->t : -1; }
 
+extern "C" int32_t fr_beam_fused_first_step(const fr_beam* bm) {
+    if (!bm) return -1;
+    return fr::root_step_fused(bm->shape, bm->trie->dev) ? 1 : 0;
+}
+
 extern "C" fr_status fr_beam_finalize(fr_beam* bm, int32_t* sids, float* scores, int32_t* items, fr_stream stream) {
     if (!bm || !sids || !scores) return FR_ERR_INVALID_ARG;
     if (bm->t != bm->shape.D) return FR_ERR_STATE;

@@ -125,6 +125,7 @@ struct StreamArgs {
     int64_t req_offset;  // index of local request 0 in the Gumbel stream
     uint64_t wait_ns;    // limit of the bounded waits that give up (abort)
     int32_t starve;      // test setting: the producer issues no copies, so the consumers' waits expire
+    int32_t slice_norm;  // fused first step: the log-sum-exp runs over the candidate slice alone
 };
 
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the finaliser of a Weyl
@@ -946,9 +947,10 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
 // the request to arrive (atomic counter, no waiting) combines them in piece
 // order, writes the root's children's scores as keys in shared memory and
 // runs the selection routine of k_select on them: top-K under the total
-// order, sort, reorder gathers and next candidate offsets.  Used at
-// temperature 0 over the full vocabulary or the SID token range when the root
-// has at most ROOT_MAX_CANDS children.
+// order, sort, reorder gathers and next candidate offsets.  Under the
+// candidate-slice normalisation nothing is streamed: one CTA per request
+// takes the log-sum-exp of the root's children alone.  Used at temperature 0
+// (every normalisation) when the root has at most ROOT_MAX_CANDS children.
 
 constexpr int ROOT_THREADS = SEL_THREADS;  // the selection routine's block size
 constexpr int ROOT_MAX_CANDS = 8192;       // root children held as keys (32 KB of shared memory)
@@ -987,6 +989,56 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
     }
     const int64_t bk = (int64_t)b * K;  // the root is slot 0
     const char* row = a.logits + bk * a.ld * ELT;
+    // the root's children: candidate slot i is child i (code order)
+    const int32_t n0 = a.node[bk];
+    int32_t clo = -1, chi = -1;
+    if (n0 >= 0 && n0 < a.trie.nodes[0]) trie_children(a.trie, 0, n0, clo, chi);
+    int32_t nch = chi - clo;
+    if (clo < 0 || nch < 0 || nch > ROOT_MAX_CANDS || a.cand_off[(int64_t)b * (K + 1)] != 0) {
+        if (tid == 0 && p == 0) set_error(a.err, FR_ERR_DEVICE);
+        nch = 0;
+    }
+    const int32_t* codes = a.trie.code[1] + clo;
+    const bool dense = a.trie.dense_c[0] != 0;
+    const int32_t tb = a.trie.tok_base[0];
+    const float sc = a.score[bk];
+    if (a.slice_norm) {
+        // candidate-slice normalisation ("Qwen-2.5-1B-RLCD-Fast", §Parallel
+        // Evaluation step 4): no row is streamed; one CTA per request takes the
+        // log-sum-exp of the root's children's logits alone
+        float m = -INFINITY, s = 0.f;
+        for (int32_t i = tid; i < nch; i += ROOT_THREADS) {
+            const float x = load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT);
+            keys[i] = __float_as_uint(x);
+            lane_add_scalar(m, s, x);
+        }
+        warp_combine(m, s);
+        if (lane == 0) wpart[warp] = make_float2(m, s);
+        __syncthreads();
+        if (warp == 0) {
+            float pm = wpart[lane].x, ps = wpart[lane].y;
+            warp_combine(pm, ps);
+            if (lane == 0) {
+                s_lse = pm + logf(ps);
+                if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
+            }
+        }
+        __syncthreads();
+        const float lse = s_lse;
+        for (int32_t i = tid; i < nch; i += ROOT_THREADS) keys[i] = float_to_key(sc + (__uint_as_float(keys[i]) - lse));
+        if (tid == 0) {
+            s_off[0] = 0;
+            s_off[1] = nch;
+            s_lo[0] = clo;
+            s_kv[0] = sl.cur.kv[bk];
+        }
+        __syncthreads();
+        const int Kp = min(K, nch);
+        const int got = block_topk<false>(SmemKeys{keys, 0u}, nch, Kp, sel, hist, red, s_misc);
+        if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
+        select_sort_emit(sl, b, 1, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+        return;
+    }
     const char* win = row + a.col0 * ELT;
     const int64_t W = a.W;
     const int64_t per = ((W + parts - 1) / parts + VE - 1) / VE * VE;
@@ -1056,21 +1108,8 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
             if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
         }
     }
-    // the root's children: candidate slot i is child i (code order)
-    const int32_t n0 = a.node[bk];
-    int32_t clo = -1, chi = -1;
-    if (n0 >= 0 && n0 < a.trie.nodes[0]) trie_children(a.trie, 0, n0, clo, chi);
-    int32_t nch = chi - clo;
-    if (clo < 0 || nch < 0 || nch > ROOT_MAX_CANDS || a.cand_off[(int64_t)b * (K + 1)] != 0) {
-        if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
-        nch = 0;
-    }
     __syncthreads();
     const float lse = s_lse;
-    const float sc = a.score[bk];
-    const int32_t* codes = a.trie.code[1] + clo;
-    const bool dense = a.trie.dense_c[0] != 0;
-    const int32_t tb = a.trie.tok_base[0];
     for (int32_t i = tid; i < nch; i += ROOT_THREADS)
         keys[i] = float_to_key(sc + (load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT) - lse));
     if (tid == 0) {
@@ -1150,8 +1189,7 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
 }
 
 bool root_step_fused(const StepShape& sh, const TrieDev& trie) {
-    return (sh.norm == FR_NORM_FULL || sh.norm == FR_NORM_SID_RANGE) && !(sh.inv_temp > 0.f) && !sh.starve &&
-           trie.nodes[1] <= ROOT_MAX_CANDS;
+    return !(sh.inv_temp > 0.f) && !sh.starve && trie.nodes[1] <= ROOT_MAX_CANDS;
 }
 
 cudaError_t root_step_setup() {
@@ -1185,6 +1223,7 @@ cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const 
     a.row_cnt = buf.row_cnt;
     a.err = buf.err;
     a.wait_ns = FR_WAIT_LIMIT_NS;
+    a.slice_norm = sh.norm == FR_NORM_CANDIDATES;
     SelectArgs sl{};
     sl.cur = cur;
     sl.nxt = buf.st[1];
@@ -1206,6 +1245,7 @@ cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const 
     parts = parts < by_len ? parts : by_len;
     parts = parts < ROOT_MAX_PARTS ? parts : ROOT_MAX_PARTS;
     parts = parts > 1 ? parts : 1;
+    if (a.slice_norm) parts = 1;  // nothing is streamed: one CTA per request
     StepLaunch L(dim3((unsigned)parts, (unsigned)sh.B), ROOT_THREADS, ROOT_MAX_CANDS * sizeof(uint32_t), s);
     return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_root_step<true>, a, sl, parts, buf.root_partial)
                                : cudaLaunchKernelEx(&L.cfg, k_root_step<false>, a, sl, parts, buf.root_partial);

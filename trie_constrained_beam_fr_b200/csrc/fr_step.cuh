@@ -83,9 +83,8 @@ cudaError_t stream_kernel_setup();  // raises the kernel's shared-memory limit
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
                           const void* logits, int64_t ld, cudaStream_t s);
 // Step 0 as one kernel (root rows + selection) instead of launch_stream +
-// launch_select: used when root_step_fused() holds (temperature 0, full
-// vocabulary or SID range, at most 8,192 root children, no wait test
-// setting).  root_step_setup raises its shared-memory
+// launch_select: used when root_step_fused() holds (temperature 0, at most
+// 8,192 root children, no wait test setting).  root_step_setup raises its shared-memory
 // limit (once per device).
 bool root_step_fused(const StepShape& sh, const TrieDev& trie);
 cudaError_t root_step_setup();

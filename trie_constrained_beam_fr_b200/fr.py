@@ -65,6 +65,7 @@ FR_FUNCS = [
     ("fr_beam_set_timing", _I32, [_VP, _I32]),
     ("fr_beam_read_timing", _I32, [_VP, _VP, _VP, _I32, _P(_I32)]),
     ("fr_beam_destroy", None, [_VP]),
+    ("fr_beam_fused_first_step", _I32, [_VP]),
     ("fr_beam_set_wait_test", _I32, [_VP, _U64, _I32]),
     ("fr_row_logsumexp_noalloc", _I32, [_VP, _I64, _I32, _I32, _I32, _VP, _VP]),
     ("fr_lmhead_init", _I32, [_VP, _I64, _I32, _I32, _I32, _I32, _I32, _P(_VP)]),
@@ -302,6 +303,14 @@ def fr_beam_set_normalization(beam, norm: int) -> None:
 def fr_beam_set_sampling(beam, temperature: float, seed: int = 0, request_offset: int = 0) -> None:
     _check(libfr().fr_beam_set_sampling(beam, float(temperature), int(seed) & 0xFFFFFFFFFFFFFFFF,
                                         int(request_offset)), "fr_beam_set_sampling")
+
+
+def fr_beam_fused_first_step(beam) -> bool:
+    """Whether the beam's first step runs as one kernel (see include/fr.h)."""
+    r = int(libfr().fr_beam_fused_first_step(beam))
+    if r < 0:
+        raise ValueError("null beam")
+    return bool(r)
 
 
 def fr_beam_set_wait_test(beam, wait_limit_ns: int = 0, starve_copies: bool = False) -> None:
