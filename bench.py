@@ -8,6 +8,9 @@ an untimed decode; each step has its own 1.9-5 GB buffer, far larger than the
 
 Metric: constrained beam candidates per second, B*K*depth per decode, summed
 over ranks (requests shard across GPUs with no collective: weak scaling).
+The timed decodes replay one decode captured in a CUDA graph from the library
+calls (`--eager` times the calls issued from Python instead); the per-kernel
+breakdown and the end-to-end leg use the calls themselves.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config serving]
     python bench.py --impl reference     # the CPU oracle on a bounded sample
@@ -47,6 +50,10 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--eager", action="store_true",
+                   help="time the library calls issued from Python instead of replays of one decode captured "
+                        "in a CUDA graph (the default; graph replay keeps host launch overhead out of small "
+                        "decodes, as a serving engine's captured decode does)")
     p.add_argument("--no-workloads", action="store_true",
                    help="with --config serving: skip the records of the other catalog-scale workloads")
     p.add_argument("--ref-requests", type=int, default=1, help="requests per reference-arm sample")
@@ -224,7 +231,9 @@ def logits_config(w: synth.Workload, args, levels) -> dict:
             "trie_levels": list(levels),
             "l2": "inputs larger than L2: one distinct %.2f GB logits buffer per step, read once"
                   % (w.B * w.K * w.V * w.elt_size / 1e9),
-            "step": "one full decode: depth beam steps + finalize"}
+            "step": "one full decode: depth beam steps + finalize",
+            "launch": "library calls from Python, stream-ordered" if getattr(args, "eager", False) else
+                      "CUDA graph replay of one decode (captured from the library calls)"}
 
 
 def lmhead_config(w: synth.Workload, args) -> dict:
@@ -620,6 +629,16 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
     for _ in range(args.warmup):
         decode()
     torch.cuda.synchronize()
+    graph = None
+    if not args.eager:
+        # one whole decode (reset, steps, finalize) as a CUDA graph: the
+        # library calls allocate nothing and never synchronise
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -629,7 +648,10 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
         # launching while the previous one drains)
         t_start.record()
         for _ in range(args.steps):
-            decode()
+            if graph is not None:
+                graph.replay()
+            else:
+                decode()
         t_end.record()
         torch.cuda.synchronize()
         barrier()
@@ -732,6 +754,7 @@ def measure_logits_workload(w: synth.Workload, args, dev, world: int, b_offset: 
                "ms_per_step": e2e_ms, "steps": args.e2e_steps}
         del host
 
+    graph = None  # release the captured decode before the buffers it names
     fr.fr_beam_destroy(beam)
     fr.fr_trie_destroy(trie)
     del bufs, out_sids, out_scores, out_items
