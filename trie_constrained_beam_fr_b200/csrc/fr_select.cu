@@ -8,15 +8,16 @@
 //
 //  k_select  per request: exact top-K of all its candidates under the strict
 //            order (score desc, slot asc) -- slot order is (parent slot,
-//            token) order -- by radix selection of order-preserving 32-bit
-//            keys (12-bit digits after skipping the bits all keys share),
-//            then a sort of the K winners on (key, ~slot); then the reorder
-//            gathers: backpointer, token, trie node, score, prefix and KV slot
-//            of every survivor, and the next step's candidate offsets.
+//            token) order -- in that order, from one histogram of
+//            order-preserving 32-bit keys (the 12 highest bits in which they
+//            differ) and a ranking of the few keys in the bins that reach the
+//            K-th; then the reorder gathers: backpointer, token, trie node,
+//            score, prefix and KV slot of every survivor, and the next step's
+//            candidate offsets.
 //  k_select_cluster  the same for requests with many candidates: a
-//            thread-block cluster per request, each CTA selecting the top-K
-//            of its slice in shared memory and the leader merging the slices'
-//            winners through distributed shared memory.
+//            thread-block cluster per request, each CTA selecting the ordered
+//            top-K of its slice in shared memory and the leader merging the
+//            slices' lists through distributed shared memory.
 //
 // Above temperature 0 ("flashrec 0.1.1 METADATA", §Serving/API: sampling
 // without replacement by Gumbel perturbation) the selection ranks the
@@ -45,11 +46,15 @@ constexpr int64_t SEL_STAGE_CAP = 16384;  // keys (64 KB of shared memory)
 
 template <bool STAGED>
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
-    extern __shared__ __align__(16) uint32_t skeys[];  // STAGED: [key_cap] the candidates as keys
+    // dynamic: the selection's scratch [SORT_CAP], then (STAGED) the
+    // candidates as keys [key_cap]
+    extern __shared__ __align__(16) unsigned long long dyn_sel[];
+    unsigned long long* tmp = dyn_sel;
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(dyn_sel + SORT_CAP);
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ int32_t s_lo[FR_MAX_K];
     __shared__ int32_t s_kv[FR_MAX_K];
-    __shared__ __align__(16) int32_t hist[HBINS];  // also the sort's scratch
+    __shared__ __align__(16) int32_t hist[HBINS];
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_misc[8];
     __shared__ uint32_t red[64];
@@ -68,51 +73,73 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
         n = 0;
     }
     const int Kp = min(K, n);
+    uint32_t va = 0xFFFFFFFFu, vo = 0u;
     int got;
     if constexpr (STAGED) {
         const float* cb = a.rank + (int64_t)b * a.cand_stride;  // 16-byte aligned
         const int nq = n >> 2;
         for (int q = tid; q < nq; q += SEL_THREADS) {
             const float4 x = __ldg(reinterpret_cast<const float4*>(cb) + q);
-            reinterpret_cast<uint4*>(skeys)[q] =
-                make_uint4(float_to_key(x.x), float_to_key(x.y), float_to_key(x.z), float_to_key(x.w));
+            const uint4 k4 = make_uint4(float_to_key(x.x), float_to_key(x.y), float_to_key(x.z), float_to_key(x.w));
+            reinterpret_cast<uint4*>(skeys)[q] = k4;
+            va &= k4.x & k4.y & k4.z & k4.w;
+            vo |= k4.x | k4.y | k4.z | k4.w;
         }
-        if (4 * nq + tid < n) skeys[4 * nq + tid] = float_to_key(__ldg(cb + 4 * nq + tid));
-        __syncthreads();
-        got = block_topk<false>(SmemKeys{skeys, 0u}, n, Kp, sel, hist, red, s_misc);
+        if (4 * nq + tid < n) {
+            const uint32_t k = float_to_key(__ldg(cb + 4 * nq + tid));
+            skeys[4 * nq + tid] = k;
+            va &= k;
+            vo |= k;
+        }
+        got = block_topk_sorted(SmemKeys{skeys, 0u}, n, Kp, va, vo, sel, tmp, hist, red, s_misc);
     } else {
-        got = block_topk<false>(GlobalCands{a.rank + (int64_t)b * a.cand_stride}, n, Kp, sel, hist, red, s_misc);
+        const GlobalCands gc{a.rank + (int64_t)b * a.cand_stride};
+        for_keys(gc, n, [&](int, uint32_t k) {
+            va &= k;
+            vo |= k;
+        });
+        got = block_topk_sorted(gc, n, Kp, va, vo, sel, tmp, hist, red, s_misc);
     }
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(a, b, live, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+    emit_survivors(a, b, live, s_off, s_lo, s_kv, Kp, sel);
 }
 
 // ---------------------------------------------------------------------------
 // Selection with one thread-block cluster per request.  Each CTA of the
 // cluster loads a contiguous slice of the request's candidates into shared
-// memory as keys and selects the slice's exact top-K with block barriers only
-// (block_topk); the union of the slices' top-Ks holds the request's top-K.
-// After one cluster barrier the leader CTA copies the CTAs' winner lists
-// (each in slot order, the slices in slot order) through distributed shared
-// memory into a pool in its own key area, a second cluster barrier releases
-// the other CTAs, and the leader selects the top-K of the pool, sorts it and
-// emits.  Every CTA runs the same two cluster barriers.
+// memory as keys and gathers a superset of the slice's top-K: the keys of its
+// histogram bins down to the one holding the slice's K-th key
+// (block_gather_top), or, when those are too many, the slice's exact top-K
+// (block_topk).  The union of the slices' sets holds the request's top-K.
+// After one cluster barrier the leader CTA copies the sets through
+// distributed shared memory into a pool in its own key area, a second cluster
+// barrier releases the other CTAs, and the leader selects the ordered top-K of
+// the pool (block_topk_sorted) and emits.  Every CTA runs the same two
+// cluster barriers.
 
 namespace cg = cooperative_groups;
 constexpr int CSEL_MAXKEYS = 40960;  // keys per CTA (160 KB of shared memory)
 
-// Dynamic shared memory of the cluster selection: a CTA's keys, and in the
-// leader later the pool of up to cs * min(K, keys per CTA) values.
-size_t csel_smem_bytes(int64_t key_cap, int cs, int K) {
-    const int64_t pool = (int64_t)cs * (K < key_cap ? K : key_cap);
-    const int64_t kb = key_cap * (int64_t)sizeof(uint32_t), pb = pool * (int64_t)sizeof(unsigned long long);
+// The cluster selection's key area: a CTA's keys, and in the leader later the
+// pool of up to cs * SORT_CAP values.  Its dynamic shared memory is the
+// selection scratch and then this area.
+size_t csel_area_bytes(int64_t key_cap, int cs) {
+    const int64_t kb = key_cap * (int64_t)sizeof(uint32_t);
+    const int64_t pb = (int64_t)cs * SORT_CAP * (int64_t)sizeof(unsigned long long);
     return (size_t)(kb > pb ? kb : pb);
+}
+size_t csel_smem_bytes(int64_t key_cap, int cs) {
+    return SORT_CAP * sizeof(unsigned long long) + csel_area_bytes(key_cap, cs);
 }
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectArgs a) {
     cg::cluster_group cl = cg::this_cluster();
-    extern __shared__ __align__(16) uint32_t keys[];  // this CTA's keys; in the leader, then the pool
-    __shared__ __align__(16) int32_t hist[HBINS];    // also the sort's scratch
+    // dynamic: the selection scratch [SORT_CAP], then this CTA's keys (in the
+    // leader, later the pool)
+    extern __shared__ __align__(16) unsigned long long dyn_csel[];
+    unsigned long long* tmp = dyn_csel;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn_csel + SORT_CAP);
+    __shared__ __align__(16) int32_t hist[HBINS];
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ int32_t s_lo[FR_MAX_K];
@@ -133,51 +160,74 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select_cluster(const SelectA
     int n = off_row[live];
     griddep_wait();
     griddep_launch_dependents();
-    if (n < 0 || (int64_t)n > a.cand_stride || (n + CS - 1) / CS > a.key_cap) {
+    if (n < 0 || (int64_t)n > a.cand_stride || (((n + CS - 1) / CS + 3) & ~3) > a.key_cap || (int64_t)CS * SORT_CAP > a.pool_cap) {
         if (tid == 0 && c == 0) set_error(a.err, FR_ERR_DEVICE);
         n = 0;
     }
     const int Kp = min(K, n);
-    const int S = (n + CS - 1) / CS;
+    const int S = ((n + CS - 1) / CS + 3) & ~3;
     const int lo = min(n, c * S), hi = min(n, lo + S);
     const int cnt = hi - lo;
-    const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;
-    int i0 = tid;
-    for (; i0 + 7 * SEL_THREADS < cnt; i0 += 8 * SEL_THREADS) {
-        float x[8];
+    const float* cb = a.rank + (int64_t)b * a.cand_stride + lo;  // 16-byte aligned: lo is a multiple of 4
+    uint32_t va = 0xFFFFFFFFu, vo = 0u;
+    const int nq = cnt >> 2;
+    for (int q0 = tid; q0 < nq; q0 += 8 * SEL_THREADS) {
+        float4 x[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = __ldg(cb + i0 + u * SEL_THREADS);
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + u * SEL_THREADS;
+            x[u] = q < nq ? __ldg(reinterpret_cast<const float4*>(cb) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) keys[i0 + u * SEL_THREADS] = float_to_key(x[u]);
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + u * SEL_THREADS;
+            if (q < nq) {
+                const uint4 k4 = make_uint4(float_to_key(x[u].x), float_to_key(x[u].y), float_to_key(x[u].z), float_to_key(x[u].w));
+                reinterpret_cast<uint4*>(keys)[q] = k4;
+                va &= k4.x & k4.y & k4.z & k4.w;
+                vo |= k4.x | k4.y | k4.z | k4.w;
+            }
+        }
     }
-    for (int i = i0; i < cnt; i += SEL_THREADS) keys[i] = float_to_key(__ldg(cb + i));
-    __syncthreads();
+    if (4 * nq + tid < cnt) {
+        const uint32_t k = float_to_key(__ldg(cb + 4 * nq + tid));
+        keys[4 * nq + tid] = k;
+        va &= k;
+        vo |= k;
+    }
     const int kc = min(Kp, cnt);
-    const int nloc = block_topk<true>(SmemKeys{keys, (uint32_t)lo}, cnt, kc, sel, hist, red, s_misc);
-    if (tid == 0) {
-        s_cnt = nloc > 0 ? nloc : 0;
-        if (nloc != kc) set_error(a.err, FR_ERR_DEVICE);
+    int m = 0;  // this slice's set, in tmp
+    if (kc > 0) {
+        const SmemKeys sk{keys, (uint32_t)lo};
+        m = block_gather_top(sk, cnt, kc, va, vo, tmp, hist, red, s_misc);
+        if (m < 0) {
+            m = block_topk(sk, cnt, kc, tmp, hist, red, s_misc);
+            if (tid == 0 && m != kc) set_error(a.err, FR_ERR_DEVICE);
+        }
     }
-    cl.sync();  // every slice's winners are in its CTA's sel
+    if (tid == 0) s_cnt = min(max(m, 0), SORT_CAP);
+    cl.sync();  // every slice's set is in its CTA's tmp
     unsigned long long* pool = reinterpret_cast<unsigned long long*>(keys);
     int P = 0;
+    uint32_t pa = 0xFFFFFFFFu, po = 0u;
     if (c == 0) {
         for (int r = 0; r < CS; ++r) {
             const int cr = *cl.map_shared_rank(&s_cnt, r);
-            if ((int64_t)P + cr > a.pool_cap) {  // cannot happen: the pool holds CS * min(K, keys per CTA)
-                if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
-                break;
+            const unsigned long long* src = cl.map_shared_rank(tmp, r);
+            for (int i = tid; i < cr; i += SEL_THREADS) {
+                const unsigned long long v = src[i];
+                pool[P + i] = v;
+                pa &= (uint32_t)(v >> 32);
+                po |= (uint32_t)(v >> 32);
             }
-            const unsigned long long* src = cl.map_shared_rank(sel, r);
-            for (int i = tid; i < cr; i += SEL_THREADS) pool[P + i] = src[i];
             P += cr;
         }
     }
-    cl.sync();  // the leader has read every list: the other CTAs may leave
+    cl.sync();  // the leader has read every set: the other CTAs may leave
     if (c != 0) return;
-    const int got = block_topk<false>(PoolVals{pool}, P, min(Kp, P), sel, hist, red, s_misc);
+    const int got = block_topk_sorted(PoolVals{pool}, P, min(Kp, P), pa, po, sel, tmp, hist, red, s_misc);
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(a, b, live, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+    emit_survivors(a, b, live, s_off, s_lo, s_kv, min(max(got, 0), Kp), sel);
 }
 
 // ---------------------------------------------------------------------------
@@ -299,21 +349,26 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
         const int64_t bound = sh.sel_bound[t];
         if (bound <= SEL_STAGE_CAP) {
             a.key_cap = (int32_t)((bound + 3) & ~(int64_t)3);
-            StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, sizeof(uint32_t) * (size_t)a.key_cap, s);
+            StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS,
+                         SORT_CAP * sizeof(unsigned long long) + sizeof(uint32_t) * (size_t)a.key_cap, s);
             return cudaLaunchKernelEx(&L.cfg, k_select<true>, a);
         }
-        StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, 0, s);
+        StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, SORT_CAP * sizeof(unsigned long long), s);
         return cudaLaunchKernelEx(&L.cfg, k_select<false>, a);
     }
-    a.key_cap = (int32_t)((sh.sel_bound[t] + cs - 1) / cs);
-    a.pool_cap = cs * (sh.K < a.key_cap ? sh.K : a.key_cap);
-    StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, csel_smem_bytes(a.key_cap, cs, sh.K), s, (unsigned)cs);
+    a.key_cap = (int32_t)(((sh.sel_bound[t] + cs - 1) / cs + 3) & ~(int64_t)3);
+    a.pool_cap = (int32_t)(csel_area_bytes(a.key_cap, cs) / sizeof(unsigned long long));
+    StepLaunch L(dim3((unsigned)(sh.B * cs)), SEL_THREADS, csel_smem_bytes(a.key_cap, cs), s, (unsigned)cs);
     return cudaLaunchKernelEx(&L.cfg, k_select_cluster, a);
 }
 
 cudaError_t select_kernel_setup() {
+    // static shared memory plus the dynamic scratch exceed the default 48 KB
+    const cudaError_t e = cudaFuncSetAttribute(k_select<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(SORT_CAP * sizeof(unsigned long long)));
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(k_select<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(SEL_STAGE_CAP * sizeof(uint32_t)));
+                                (int)(SORT_CAP * sizeof(unsigned long long) + SEL_STAGE_CAP * sizeof(uint32_t)));
 }
 
 int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {
@@ -333,14 +388,14 @@ int select_cluster_size(int32_t B, int32_t K, int64_t bound, int32_t sms) {
     const int cs = need > fill ? need : fill;
     if (cs < 2 || (int64_t)B * cs > sms) return 0;
     if (cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)csel_smem_bytes(CSEL_MAXKEYS, 8, FR_MAX_K)) != cudaSuccess) {
+                             (int)csel_smem_bytes(CSEL_MAXKEYS, 8)) != cudaSuccess) {
         (void)cudaGetLastError();
         return 0;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(B * cs));
     cfg.blockDim = dim3(SEL_THREADS);
-    cfg.dynamicSmemBytes = csel_smem_bytes((bound + cs - 1) / cs, cs, K);
+    cfg.dynamicSmemBytes = csel_smem_bytes(((bound + cs - 1) / cs + 3) & ~(int64_t)3, cs);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;

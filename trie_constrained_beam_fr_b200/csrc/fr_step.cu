@@ -963,7 +963,8 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
     constexpr int ELT = BF16 ? 2 : 4;
     constexpr int64_t VE = 16 / ELT;
     extern __shared__ __align__(16) uint32_t keys[];  // [ROOT_MAX_CANDS]
-    __shared__ __align__(16) int32_t hist[HBINS];    // also the sort's scratch
+    __shared__ __align__(16) int32_t hist[HBINS];
+    __shared__ __align__(16) unsigned long long tmp[SORT_CAP];
     __shared__ __align__(16) unsigned long long sel[FR_MAX_K];
     __shared__ int32_t s_off[2];
     __shared__ int32_t s_lo[1];
@@ -984,7 +985,7 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         // no beam at all: the request's next state is all dead
         if (tid == 0) s_off[0] = s_off[1] = 0;
         __syncthreads();
-        select_sort_emit(sl, b, 0, s_off, s_lo, s_kv, 0, sel, reinterpret_cast<unsigned long long*>(hist));
+        emit_survivors(sl, b, 0, s_off, s_lo, s_kv, 0, sel);
         return;
     }
     const int64_t bk = (int64_t)b * K;  // the root is slot 0
@@ -1025,7 +1026,13 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         }
         __syncthreads();
         const float lse = s_lse;
-        for (int32_t i = tid; i < nch; i += ROOT_THREADS) keys[i] = float_to_key(sc + (__uint_as_float(keys[i]) - lse));
+        uint32_t va = 0xFFFFFFFFu, vo = 0u;
+        for (int32_t i = tid; i < nch; i += ROOT_THREADS) {
+            const uint32_t k = float_to_key(sc + (__uint_as_float(keys[i]) - lse));
+            keys[i] = k;
+            va &= k;
+            vo |= k;
+        }
         if (tid == 0) {
             s_off[0] = 0;
             s_off[1] = nch;
@@ -1034,9 +1041,9 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         }
         __syncthreads();
         const int Kp = min(K, nch);
-        const int got = block_topk<false>(SmemKeys{keys, 0u}, nch, Kp, sel, hist, red, s_misc);
+        const int got = block_topk_sorted(SmemKeys{keys, 0u}, nch, Kp, va, vo, sel, tmp, hist, red, s_misc);
         if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-        select_sort_emit(sl, b, 1, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+        emit_survivors(sl, b, 1, s_off, s_lo, s_kv, Kp, sel);
         return;
     }
     const char* win = row + a.col0 * ELT;
@@ -1087,9 +1094,13 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
     }
     __syncthreads();
     if (!s_last) return;
-    // the last piece of the row has arrived: combine the pieces in order
+    // the last piece of the row has arrived: warp 0 combines the pieces in
+    // order while the other warps fetch the root's children's logits
     __threadfence();
-    if (warp == 0) {
+    if (warp != 0) {
+        for (int32_t i = tid - 32; i < nch; i += ROOT_THREADS - 32)
+            keys[i] = __float_as_uint(load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT));
+    } else {
         float M = -INFINITY, S = 0.f;
         for (int base = 0; base < parts; base += 32) {
             const int g = base + lane;
@@ -1108,10 +1119,6 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
             if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
         }
     }
-    __syncthreads();
-    const float lse = s_lse;
-    for (int32_t i = tid; i < nch; i += ROOT_THREADS)
-        keys[i] = float_to_key(sc + (load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT) - lse));
     if (tid == 0) {
         s_off[0] = 0;
         s_off[1] = nch;
@@ -1119,10 +1126,20 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         s_kv[0] = sl.cur.kv[bk];
     }
     __syncthreads();
+    // the candidates' keys (each thread rewrites the entries it reads; the
+    // selection's first barrier publishes them)
+    const float lse = s_lse;
+    uint32_t va = 0xFFFFFFFFu, vo = 0u;
+    for (int32_t i = tid; i < nch; i += ROOT_THREADS) {
+        const uint32_t k = float_to_key(sc + (__uint_as_float(keys[i]) - lse));
+        keys[i] = k;
+        va &= k;
+        vo |= k;
+    }
     const int Kp = min(K, nch);
-    const int got = block_topk<false>(SmemKeys{keys, 0u}, nch, Kp, sel, hist, red, s_misc);
+    const int got = block_topk_sorted(SmemKeys{keys, 0u}, nch, Kp, va, vo, sel, tmp, hist, red, s_misc);
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
-    select_sort_emit(sl, b, 1, s_off, s_lo, s_kv, Kp, sel, reinterpret_cast<unsigned long long*>(hist));
+    emit_survivors(sl, b, 1, s_off, s_lo, s_kv, Kp, sel);
 }
 
 }  // namespace

@@ -20,9 +20,15 @@ namespace {
 constexpr int SEL_THREADS = 1024;
 constexpr int HBITS = 12;
 constexpr int HBINS = 1 << HBITS;
+// The one-pass selection (block_topk_sorted) places at most SORT_CAP
+// candidates, each by comparisons within its histogram bin of at most
+// RANK_CAP keys; past either bound it falls back to the radix selection.
+constexpr int SORT_CAP = 2048;
+constexpr int RANK_CAP = 128;
 static_assert(HBINS == 4 * SEL_THREADS, "each thread owns four histogram bins");
 static_assert(FR_MAX_K <= SEL_THREADS, "one thread per beam slot");
 static_assert(HBINS * sizeof(int32_t) >= FR_MAX_K * sizeof(unsigned long long), "histogram doubles as sort scratch");
+static_assert(SORT_CAP >= FR_MAX_K, "the sort scratch holds K values");
 
 struct SelectArgs {
     StateDev cur, nxt;
@@ -38,8 +44,11 @@ struct SelectArgs {
     int32_t pool_cap;  // cluster select: values the leader's pool holds
 };
 
-__device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t* out_or) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// AND and OR of one word per thread over the block, both returned to every
+// thread.  One barrier: red [64] may be written again only after a later one.
+__device__ __forceinline__ void block_and_or(uint32_t v_and, uint32_t v_or, uint32_t* red, uint32_t& all_and,
+                                             uint32_t& all_or) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     v_and = __reduce_and_sync(0xffffffffu, v_and);
     v_or = __reduce_or_sync(0xffffffffu, v_or);
     if (lane == 0) {
@@ -47,15 +56,24 @@ __device__ __forceinline__ uint32_t block_and_or(uint32_t v_and, uint32_t v_or, 
         red[32 + warp] = v_or;
     }
     __syncthreads();
-    const int nw = blockDim.x >> 5;
-    uint32_t a = 0xFFFFFFFFu, o = 0u;
-    for (int w = 0; w < nw; ++w) {
-        a &= red[w];
-        o |= red[32 + w];
-    }
+    all_and = __reduce_and_sync(0xffffffffu, lane < nw ? red[lane] : 0xFFFFFFFFu);
+    all_or = __reduce_or_sync(0xffffffffu, lane < nw ? red[32 + lane] : 0u);
+}
+
+// Exclusive scan of one int per thread across the block (blockDim.x a
+// multiple of 32, at most 1024) for the last scan a kernel makes: one barrier,
+// and none after it, so a block must call it at most once.  *total receives
+// the block sum.
+__device__ __forceinline__ int block_excl_scan_once(int v, int* total) {
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int incl = warp_incl_scan(v);
+    if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    *out_or = o;
-    return a;
+    const int ws = lane < nw ? wsum[lane] : 0;
+    const int wi = warp_incl_scan(ws);
+    *total = __shfl_sync(0xffffffffu, wi, 31);
+    return __shfl_sync(0xffffffffu, wi - ws, warp) + incl - v;
 }
 
 // Next step's candidate offsets of request b: exclusive scan over slots of
@@ -165,45 +183,63 @@ __device__ __forceinline__ void load_parents(const SelectArgs& a, int b, int liv
     }
 }
 
-__device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int32_t* s_off, const int32_t* s_lo,
-                                 const int32_t* s_kv, int Kp, unsigned long long* sel, unsigned long long* scratch) {
-    const int tid = threadIdx.x;
+// Writes request b's next state from its Kp winners, sel[0..Kp) in order
+// (descending value): thread j takes survivor j -- its parent slot (the last k
+// with s_off[k] <= its candidate slot), trie node, token, score, KV slot and
+// prefix -- and, unless this is the last step, the next step's candidate
+// offsets (an exclusive scan of the survivors' child counts).  The global
+// loads a survivor needs (its node's children, its token code, its parent's
+// prefix) are issued together, before its stores.  All threads of the block
+// (blockDim.x >= K) call it.
+__device__ void emit_survivors(const SelectArgs& a, int b, int live, const int32_t* s_off, const int32_t* s_lo,
+                               const int32_t* s_kv, int Kp, const unsigned long long* sel) {
+    const int j = threadIdx.x;
     const int K = a.K, D = a.D, t = a.t;
-    sort_desc_u64(sel, scratch, Kp);
-
-    // emit survivors (thread j = slot j)
-    const int j = tid;
-    int32_t child = -1;
+    const bool more = t + 1 < D;
+    int32_t child = -1, tok = -1, k = 0, nchild = 0;
+    uint32_t key = 0u;
+    int32_t slot = 0;
+    if (j < Kp) {
+        const unsigned long long v = sel[j];
+        key = (uint32_t)(v >> 32);
+        slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
+        int lo = 0, hi = live - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
+        }
+        k = lo;
+        if (s_lo[k] >= 0) {
+            const int32_t c = s_lo[k] + (slot - s_off[k]);
+            if (c >= 0 && c < a.trie.nodes[t + 1]) child = c;
+        }
+        if (child >= 0) {
+            if (more) {
+                int32_t clo, chi;
+                trie_children(a.trie, t + 1, child, clo, chi);
+                nchild = chi - clo;
+            }
+            tok = a.trie.tok_base[t] + trie_child_code(a.trie, t, child);
+        } else {
+            set_error(a.err, FR_ERR_DEVICE);
+        }
+    }
     if (j < K) {
         const int64_t oj = (int64_t)b * K + j;
         if (j < Kp) {
-            const unsigned long long v = sel[j];
-            const uint32_t key = (uint32_t)(v >> 32);
-            const int32_t slot = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
-            int lo = 0, hi = live - 1;  // parent: last k with s_off[k] <= slot
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_off[mid] <= slot) lo = mid; else hi = mid - 1;
-            }
-            const int k = lo;
             const int64_t ok = (int64_t)b * K + k;
-            int32_t tok = -1;
-            if (s_lo[k] >= 0) {
-                child = s_lo[k] + (slot - s_off[k]);
-                if (child >= 0 && child < a.trie.nodes[t + 1]) {
-                    tok = a.trie.tok_base[t] + trie_child_code(a.trie, t, child);
-                } else {
-                    child = -1;
-                }
-            }
-            if (child < 0) set_error(a.err, FR_ERR_DEVICE);
+            int32_t pre[FR_MAX_DEPTH];
+#pragma unroll
+            for (int l = 0; l < FR_MAX_DEPTH; ++l) pre[l] = (l < t) ? __ldg(a.cur.prefix + ok * D + l) : -1;
+            const float sc = (a.rank == a.cand) ? key_to_float(key) : __ldg(a.cand + (int64_t)b * a.cand_stride + slot);
             a.nxt.node[oj] = child;
-            a.nxt.score[oj] = (a.rank == a.cand) ? key_to_float(key) : a.cand[(int64_t)b * a.cand_stride + slot];
+            a.nxt.score[oj] = sc;
             a.nxt.kv[oj] = s_kv[k];
             a.parent_out[oj] = k;
             a.token_out[oj] = tok;
-            for (int l = 0; l < D; ++l)
-                a.nxt.prefix[oj * D + l] = (l < t) ? a.cur.prefix[ok * D + l] : (l == t ? tok : -1);
+#pragma unroll
+            for (int l = 0; l < FR_MAX_DEPTH; ++l)
+                if (l < D) a.nxt.prefix[oj * D + l] = (l < t) ? pre[l] : (l == t ? tok : -1);
         } else {
             a.nxt.node[oj] = -1;
             a.nxt.score[oj] = -INFINITY;
@@ -213,21 +249,13 @@ __device__ void select_sort_emit(const SelectArgs& a, int b, int live, const int
             for (int l = 0; l < D; ++l) a.nxt.prefix[oj * D + l] = -1;
         }
     }
-    if (tid == 0) a.nxt.live[b] = Kp;
-    if (t + 1 < D) {
-        // node ids of the survivors are in registers of threads 0..Kp-1
-        const int jj = threadIdx.x;
-        int cnt = 0;
-        if (jj < Kp && child >= 0) {
-            int32_t lo, hi;
-            trie_children(a.trie, t + 1, child, lo, hi);
-            cnt = hi - lo;
-        }
+    if (j == 0) a.nxt.live[b] = Kp;
+    if (more) {
         int tot;
-        const int e = block_excl_scan(cnt, &tot);
+        const int e = block_excl_scan_once(nchild, &tot);
         int32_t* row = a.nxt.cand_off + (int64_t)b * (K + 1);
-        if (jj < K) row[jj] = e;
-        if (jj == 0) row[K] = tot;
+        if (j < K) row[j] = e;
+        if (j == 0) row[K] = tot;
     }
 }
 
@@ -261,7 +289,7 @@ struct SmemKeys {  // a contiguous slice of them, as keys in shared memory, slot
     }
     __device__ __forceinline__ unsigned long long val(int i) const { return val_of(i, keys[i]); }
 };
-struct PoolVals {  // values already formed, in slot order
+struct PoolVals {  // values already formed
     static constexpr bool QUADS = false;
     const unsigned long long* pool;
     __device__ __forceinline__ uint32_t key(int i) const { return (uint32_t)(pool[i] >> 32); }
@@ -270,46 +298,50 @@ struct PoolVals {  // values already formed, in slot order
 };
 
 // Calls f(i, key(i)) for the indices i in [0, n) this thread owns (which ones
-// depends on the access width), with eight independent loads in flight per
-// thread.  The calls' order is not index order.
+// depends on the access width), loading several keys before using any: eight
+// 16-byte groups of four from global memory (a pass over n keys takes
+// ceil(n / (32 * SEL_THREADS)) memory round trips), four single keys from
+// shared memory (a shorter body: these kernels run their code once, so its
+// size costs instruction fetches).  The calls' order is not index order.
 template <class Vals, class F>
 __device__ __forceinline__ void for_keys(const Vals& vals, int n, F&& f) {
     const int tid = threadIdx.x;
     if constexpr (Vals::QUADS) {
         const int nq = n >> 2;
-        int q0 = tid;
-        for (; q0 + 7 * SEL_THREADS < nq; q0 += 8 * SEL_THREADS) {
+        for (int q0 = tid; q0 < nq; q0 += 8 * SEL_THREADS) {
             uint4 k4[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) k4[u] = vals.key4(q0 + u * SEL_THREADS);
+            for (int u = 0; u < 8; ++u) {
+                const int q = q0 + u * SEL_THREADS;
+                k4[u] = q < nq ? vals.key4(q) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int i = (q0 + u * SEL_THREADS) * 4;
-                f(i, k4[u].x);
-                f(i + 1, k4[u].y);
-                f(i + 2, k4[u].z);
-                f(i + 3, k4[u].w);
+                const int q = q0 + u * SEL_THREADS;
+                if (q < nq) {
+                    f(4 * q, k4[u].x);
+                    f(4 * q + 1, k4[u].y);
+                    f(4 * q + 2, k4[u].z);
+                    f(4 * q + 3, k4[u].w);
+                }
             }
-        }
-        for (int q = q0; q < nq; q += SEL_THREADS) {
-            const uint4 k4 = vals.key4(q);
-            f(4 * q, k4.x);
-            f(4 * q + 1, k4.y);
-            f(4 * q + 2, k4.z);
-            f(4 * q + 3, k4.w);
         }
         const int i = 4 * nq + tid;  // the last n mod 4
         if (i < n) f(i, vals.key(i));
     } else {
-        int i0 = tid;
-        for (; i0 + 7 * SEL_THREADS < n; i0 += 8 * SEL_THREADS) {
-            uint32_t k8[8];
+        for (int i0 = tid; i0 < n; i0 += 4 * SEL_THREADS) {
+            uint32_t k8[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) k8[u] = vals.key(i0 + u * SEL_THREADS);
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * SEL_THREADS;
+                k8[u] = i < n ? vals.key(i) : 0u;
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) f(i0 + u * SEL_THREADS, k8[u]);
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * SEL_THREADS;
+                if (i < n) f(i, k8[u]);
+            }
         }
-        for (int i = i0; i < n; i += SEL_THREADS) f(i, vals.key(i));
     }
 }
 
@@ -320,18 +352,15 @@ __device__ __forceinline__ void for_keys(const Vals& vals, int n, F&& f) {
 // bits every key shares); the winners are every key > T and the lowest-index
 // keys == T.  The search stops early once the bin holding the Kp-th key holds
 // exactly the keys still needed: T is then that bin's lowest value, and the
-// winners are the keys >= T.  ORDERED: they are written in index (slot) order -- each warp
-// owns a contiguous block of indices and counts its keys above and at T
-// (ballots), one scan over the warps gives each warp its output offset, and a
-// second sweep writes.  Otherwise in any order, in one sweep (atomic
-// positions; when not all the keys equal to T win, their lowest indices are
-// found by ranking them, or, past SEL_THREADS of them, by block scans in index
-// order).  All threads of the block call it; scratch:
+// winners are the keys >= T.  They are written in any order, in one sweep
+// (atomic positions; when not all the keys equal to T win, their lowest
+// indices are found by ranking them, or, past SEL_THREADS of them, by block
+// scans in index order).  All threads of the block call it; scratch:
 // hist [HBINS], red [64], s_misc [8].
-template <bool ORDERED, class Vals>
+template <class Vals>
 __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* out, int32_t* hist, uint32_t* red,
                           int32_t* s_misc) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     if (Kp <= 0 || n <= 0) return 0;
     uint32_t T = 0u;
     int eq_needed = n;  // Kp == n: every value wins (all keys are >= 0)
@@ -342,8 +371,8 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
             va &= k;
             vo |= k;
         });
-        uint32_t VO;
-        const uint32_t VA = block_and_or(va, vo, red, &VO);
+        uint32_t VA, VO;
+        block_and_or(va, vo, red, VA, VO);
         const uint32_t diff = VA ^ VO;
         if (diff == 0u) {
             T = VA;
@@ -396,7 +425,7 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
             eq_needed = krem;
         }
     }
-    if constexpr (!ORDERED) {
+    {
         if (tid == 0) {
             s_misc[3] = 0;
             s_misc[4] = 0;
@@ -454,71 +483,128 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
         __syncthreads();
         return s_misc[3];
     }
-    // collect in index order
+}
+
+// The keys of the bins at and above the one holding the Kp-th largest key
+// (0 < Kp <= n, Kp <= FR_MAX_K), as values in tmp[0..M), grouped by bin,
+// highest bin first; returns M.  va / vo: this thread's AND / OR over the keys
+// it has read (every key read by some thread).  One histogram pass over the
+// 12 highest bits in which the keys differ gives every bin the number of keys
+// above it (hist[d] then holds where bin d's group ends, and the next lower
+// bin's starts; the digit is (key >> s_misc[3]) & s_misc[4]).  s_misc[6] = 1
+// when tmp[0..M) is already in order (every key the same: the Kp lowest slots).
+// Returns -1 when those bins hold more than SORT_CAP keys or one of them more
+// than RANK_CAP.  All threads of the block (blockDim.x == SEL_THREADS) call
+// it; the keys must be readable by all of them on entry; it ends with a
+// barrier.  Scratch: hist [HBINS], tmp [SORT_CAP], red [64], s_misc [8].
+template <class Vals>
+__device__ int block_gather_top(const Vals& vals, int n, int Kp, uint32_t va, uint32_t vo, unsigned long long* tmp,
+                                int32_t* hist, uint32_t* red, int32_t* s_misc) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = SEL_THREADS / 32;
-    const int per = (((n + NW - 1) / NW) + 31) & ~31;
-    const int beg = min(n, warp * per), end = min(n, beg + per);
-    constexpr int CB = 8;  // 32-wide rows per batch: CB independent loads in flight per lane
-    int cgt = 0, ceq = 0;
-    for (int j = beg; j < end; j += 32 * CB) {
-        uint32_t k8[CB];
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const int i = j + u * 32 + lane;
-            k8[u] = i < end ? vals.key(i) : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const bool in = j + u * 32 + lane < end;
-            cgt += __popc(__ballot_sync(0xffffffffu, in && k8[u] > T));
-            ceq += __popc(__ballot_sync(0xffffffffu, in && k8[u] == T));
-        }
+    reinterpret_cast<int4*>(hist)[tid] = make_int4(0, 0, 0, 0);
+    if (tid == 0) {
+        s_misc[5] = 0;
+        s_misc[6] = 0;
     }
-    if (lane == 0) {
-        red[warp] = (uint32_t)cgt;
-        red[NW + warp] = (uint32_t)ceq;
+    uint32_t VA, VO;
+    block_and_or(va, vo, red, VA, VO);  // its barrier also publishes the zeroed histogram
+    const uint32_t diff = VA ^ VO;
+    if (diff == 0u) {
+        for (int j = tid; j < Kp; j += SEL_THREADS) tmp[j] = vals.val_of(j, VA);
+        if (tid == 0) s_misc[6] = 1;
+        __syncthreads();
+        return Kp;
+    }
+    const int lo = 32 - __clz(diff);  // bits >= lo are the same in every key
+    const int width = min(HBITS, lo), shift = lo - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    for_keys(vals, n, [&](int, uint32_t k) { atomicAdd(&hist[(k >> shift) & dmask], 1); });
+    __syncthreads();
+    // keys above each bin: thread t owns bins 4t .. 4t+3, higher threads own
+    // higher bins; a scan over the threads from the top
+    const int4 h4 = reinterpret_cast<const int4*>(hist)[tid];
+    const int hq[4] = {h4.x, h4.y, h4.z, h4.w};
+    const int tsum = h4.x + h4.y + h4.z + h4.w;
+    const int incl = warp_incl_scan(tsum);
+    if (lane == 31) red[warp] = (uint32_t)incl;
+    __syncthreads();
+    const int ws = lane < NW ? (int)red[lane] : 0;
+    const int wi = warp_incl_scan(ws);
+    const int total = __shfl_sync(0xffffffffu, wi, 31);
+    const int below = __shfl_sync(0xffffffffu, wi - ws, warp) + incl;  // keys in bins of threads <= tid
+    int cum = total - below;
+    int off[4];
+    bool big = false;
+#pragma unroll
+    for (int q = 3; q >= 0; --q) {
+        off[q] = cum;
+        if (cum < Kp) {  // a bin at or above the one holding the Kp-th key
+            if (cum + hq[q] >= Kp) {
+                s_misc[0] = 4 * tid + q;
+                s_misc[1] = cum;
+                s_misc[2] = hq[q];
+            }
+            if (hq[q] > RANK_CAP) big = true;
+        }
+        cum += hq[q];
+    }
+    if (big) s_misc[5] = 1;
+    reinterpret_cast<int4*>(hist)[tid] = make_int4(off[0], off[1], off[2], off[3]);
+    __syncthreads();
+    const int bstar = s_misc[0];
+    const int M = s_misc[1] + s_misc[2];
+    if (M > SORT_CAP || s_misc[5] != 0) return -1;
+    const uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
+    const uint32_t floor_key = prefix | ((uint32_t)bstar << shift);  // keys >= it: bins >= bstar
+    for_keys(vals, n, [&](int i, uint32_t k) {
+        if (k >= floor_key) {
+            const int p = atomicAdd(&hist[(k >> shift) & dmask], 1);
+            if (p < M) tmp[p] = vals.val_of(i, k);  // always: the keys are the ones counted
+        }
+    });
+    if (tid == 0) {
+        s_misc[3] = shift;
+        s_misc[4] = (int32_t)dmask;
     }
     __syncthreads();
-    if (warp == 0) {
-        const int g = lane < NW ? (int)red[lane] : 0, e = lane < NW ? (int)red[NW + lane] : 0;
-        const int gi = warp_incl_scan(g), ei = warp_incl_scan(e);
-        if (lane < NW) {
-            red[lane] = (uint32_t)(gi - g);
-            red[NW + lane] = (uint32_t)(ei - e);
+    return M;
+}
+
+// Exact top-Kp (0 < Kp <= n, Kp <= FR_MAX_K) of the n values, in order
+// (descending value: key descending, slot ascending), into out[0..Kp);
+// returns how many were written (Kp unless something is inconsistent).  The
+// values block_gather_top gathers each go to their bin's first place plus the
+// number of larger values in their bin (at most RANK_CAP comparisons); when it
+// declines, the radix selection (block_topk) finds the winners and they are
+// sorted.  Same calling rules and scratch as block_gather_top.
+template <class Vals>
+__device__ int block_topk_sorted(const Vals& vals, int n, int Kp, uint32_t va, uint32_t vo, unsigned long long* out,
+                                 unsigned long long* tmp, int32_t* hist, uint32_t* red, int32_t* s_misc) {
+    const int tid = threadIdx.x;
+    if (Kp <= 0 || n <= 0) return 0;
+    const int M = block_gather_top(vals, n, Kp, va, vo, tmp, hist, red, s_misc);
+    if (M >= 0) {
+        if (s_misc[6]) {
+            for (int j = tid; j < Kp; j += SEL_THREADS) out[j] = tmp[j];
+        } else {
+            const int shift = s_misc[3];
+            const uint32_t dmask = (uint32_t)s_misc[4];
+            for (int p = tid; p < M; p += SEL_THREADS) {
+                const unsigned long long v = tmp[p];
+                const int d = (int)(((uint32_t)(v >> 32) >> shift) & dmask);
+                const int beg = d < (int)dmask ? hist[d + 1] : 0, end = min(hist[d], M);
+                int r = 0;
+                for (int q = beg; q < end; ++q) r += tmp[q] > v;
+                if (beg + r < Kp) out[beg + r] = v;
+            }
         }
-        if (lane == 31) {
-            s_misc[6] = gi;
-            s_misc[7] = ei;
-        }
+        __syncthreads();
+        return Kp;
     }
-    __syncthreads();
-    int gbase = (int)red[warp], ebase = (int)red[NW + warp];
-    const int total = s_misc[6] + min(s_misc[7], eq_needed);
-    const unsigned lt = (1u << lane) - 1u;
-    for (int j = beg; j < end; j += 32 * CB) {
-        unsigned long long v8[CB];
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const int i = j + u * 32 + lane;
-            v8[u] = i < end ? vals.val(i) : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const bool in = j + u * 32 + lane < end;
-            const uint32_t k = (uint32_t)(v8[u] >> 32);
-            const bool g = in && k > T, e = in && k == T;
-            const unsigned bg = __ballot_sync(0xffffffffu, g), be = __ballot_sync(0xffffffffu, e);
-            const int gb = gbase + __popc(bg & lt), eb = ebase + __popc(be & lt);
-            int pos = -1;
-            if (g) pos = gb + min(eb, eq_needed);
-            else if (e && eb < eq_needed) pos = gb + eb;
-            if (pos >= 0 && pos < Kp) out[pos] = v8[u];
-            gbase += __popc(bg);
-            ebase += __popc(be);
-        }
-    }
-    __syncthreads();
-    return total;
+    const int got = block_topk(vals, n, Kp, out, hist, red, s_misc);
+    sort_desc_u64(out, tmp, got);
+    return got;
 }
 
 }  // namespace
