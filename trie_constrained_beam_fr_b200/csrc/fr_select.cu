@@ -40,17 +40,22 @@ namespace {
 
 // STAGED: the request's candidates (at most key_cap of them) are read once
 // into shared memory as keys and every pass of the selection reads them from
-// there; otherwise every pass reads them from global memory (L2).  Two
-// instantiations so that the global-memory version keeps its own code.
+// there; otherwise the passes read them from global memory (L2), and with up
+// to SEL_DIGIT_CAP candidates the histogram pass records each one's bin in
+// shared memory (16 bits) so that the gathering pass reads only the gathered
+// keys again.  Two instantiations so that the global-memory version keeps its
+// own code.
 constexpr int64_t SEL_STAGE_CAP = 16384;  // keys (64 KB of shared memory)
+constexpr int64_t SEL_DIGIT_CAP = 65536;  // bins (128 KB of shared memory)
 
 template <bool STAGED>
 __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     // dynamic: the selection's scratch [SORT_CAP], then (STAGED) the
-    // candidates as keys [key_cap]
+    // candidates as keys [key_cap], or (key_cap > 0, not STAGED) their bins
     extern __shared__ __align__(16) unsigned long long dyn_sel[];
     unsigned long long* tmp = dyn_sel;
     uint32_t* skeys = reinterpret_cast<uint32_t*>(dyn_sel + SORT_CAP);
+    uint16_t* digits = (!STAGED && a.key_cap > 0) ? reinterpret_cast<uint16_t*>(dyn_sel + SORT_CAP) : nullptr;
     __shared__ int32_t s_off[FR_MAX_K + 1];
     __shared__ int32_t s_lo[FR_MAX_K];
     __shared__ int32_t s_kv[FR_MAX_K];
@@ -68,7 +73,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
     griddep_launch_dependents();
     __syncthreads();
     int n = s_off[live];
-    if (n < 0 || (int64_t)n > a.cand_stride || (STAGED && n > a.key_cap)) {
+    if (n < 0 || (int64_t)n > a.cand_stride || ((STAGED || digits) && n > a.key_cap)) {
         if (tid == 0) set_error(a.err, FR_ERR_DEVICE);
         n = 0;
     }
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) k_select(const SelectArgs a) {
             va &= k;
             vo |= k;
         });
-        got = block_topk_sorted(gc, n, Kp, va, vo, sel, tmp, hist, red, s_misc);
+        got = block_topk_sorted(gc, n, Kp, va, vo, sel, tmp, hist, red, s_misc, digits);
     }
     if (tid == 0 && got != Kp) set_error(a.err, FR_ERR_DEVICE);
     emit_survivors(a, b, live, s_off, s_lo, s_kv, Kp, sel);
@@ -353,7 +358,9 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
                          SORT_CAP * sizeof(unsigned long long) + sizeof(uint32_t) * (size_t)a.key_cap, s);
             return cudaLaunchKernelEx(&L.cfg, k_select<true>, a);
         }
-        StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS, SORT_CAP * sizeof(unsigned long long), s);
+        a.key_cap = bound <= SEL_DIGIT_CAP ? (int32_t)((bound + 7) & ~(int64_t)7) : 0;
+        StepLaunch L(dim3((unsigned)sh.B), SEL_THREADS,
+                     SORT_CAP * sizeof(unsigned long long) + sizeof(uint16_t) * (size_t)a.key_cap, s);
         return cudaLaunchKernelEx(&L.cfg, k_select<false>, a);
     }
     a.key_cap = (int32_t)(((sh.sel_bound[t] + cs - 1) / cs + 3) & ~(int64_t)3);
@@ -365,7 +372,7 @@ cudaError_t launch_select(const StepShape& sh, const StepBuffers& buf, const Tri
 cudaError_t select_kernel_setup() {
     // static shared memory plus the dynamic scratch exceed the default 48 KB
     const cudaError_t e = cudaFuncSetAttribute(k_select<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(SORT_CAP * sizeof(unsigned long long)));
+                                               (int)(SORT_CAP * sizeof(unsigned long long) + SEL_DIGIT_CAP * sizeof(uint16_t)));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(k_select<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(SORT_CAP * sizeof(unsigned long long) + SEL_STAGE_CAP * sizeof(uint32_t)));

@@ -36,6 +36,7 @@
 // a test setting gives) the kernel records FR_ERR_DEVICE in the beam's status
 // word and returns, with no copy in flight.
 #include <cuda_bf16.h>
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -45,6 +46,8 @@
 
 namespace fr {
 namespace {
+
+namespace cg = cooperative_groups;
 
 // Consumer warps reduce the staged chunks.  The bf16 reduction is bound by
 // the latency of its exponentials (one MUFU ex2 per element), not by their
@@ -941,25 +944,27 @@ __global__ void __launch_bounds__(256) k_slice_candidates(const StreamArgs a) {
 // root's children.  Run as the two general kernels, the streaming kernel's
 // pipeline never fills and the selection pays its own launch; here one kernel
 // does the whole step: the root row of request b is cut into `parts` equal
-// pieces, one CTA each (16-byte vectors, a batch of ROOT_VPL per thread in
-// flight, each batch's maximum first and then its exponent sum against the
-// running maximum); each CTA leaves its (max, scaled sum) and the last CTA of
-// the request to arrive (atomic counter, no waiting) combines them in piece
-// order, writes the root's children's scores as keys in shared memory and
-// runs the selection routine of k_select on them: top-K under the total
-// order, sort, reorder gathers and next candidate offsets.  Under the
+// pieces, one CTA each, the CTAs of a request forming one thread-block
+// cluster (16-byte vectors, a batch of ROOT_VPL per thread in flight, each
+// batch's maximum first and then its exponent sum against the running
+// maximum); each CTA stores its (max, scaled sum) into the first CTA's shared
+// memory (distributed shared memory), and after one cluster barrier the first
+// CTA combines them in piece order, writes the root's children's scores (their
+// logits loaded before its piece) as keys in shared memory and runs the
+// selection routine of k_select on them: the ordered top-K, reorder gathers
+// and next candidate offsets.  Under the
 // candidate-slice normalisation nothing is streamed: one CTA per request
 // takes the log-sum-exp of the root's children alone.  Used at temperature 0
 // (every normalisation) when the root has at most ROOT_MAX_CANDS children.
 
 constexpr int ROOT_THREADS = SEL_THREADS;  // the selection routine's block size
 constexpr int ROOT_MAX_CANDS = 8192;       // root children held as keys (32 KB of shared memory)
-constexpr int ROOT_MAX_PARTS = 64;         // pieces per root row
+constexpr int ROOT_MAX_PARTS = 8;          // pieces per root row: the portable cluster size
 constexpr int ROOT_VPL = 4;                // 16-byte vectors per thread per batch
 
 template <bool BF16>
 __global__ void __launch_bounds__(ROOT_THREADS, 1)
-    k_root_step(const StreamArgs a, const SelectArgs sl, int32_t parts, float2* __restrict__ rpart) {
+    k_root_step(const StreamArgs a, const SelectArgs sl, int32_t parts) {
     constexpr int ELT = BF16 ? 2 : 4;
     constexpr int64_t VE = 16 / ELT;
     extern __shared__ __align__(16) uint32_t keys[];  // [ROOT_MAX_CANDS]
@@ -972,8 +977,8 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
     __shared__ uint32_t red[64];
     __shared__ int32_t s_misc[8];
     __shared__ float2 wpart[ROOT_THREADS / 32];
+    __shared__ float2 s_pieces[ROOT_MAX_PARTS];  // the first CTA's: every piece's (max, scaled sum)
     __shared__ float s_lse;
-    __shared__ int32_t s_last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int p = blockIdx.x, b = blockIdx.y;
     const int K = a.K;
@@ -1046,6 +1051,10 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         emit_survivors(sl, b, 1, s_off, s_lo, s_kv, Kp, sel);
         return;
     }
+    // the first CTA's threads each load one of the root's first ROOT_THREADS
+    // children's logits now, so that they arrive while the row streams
+    float child_x = 0.f;
+    if (p == 0 && tid < nch) child_x = load_elem(row, tb + (dense ? tid : __ldg(codes + tid)), ELT);
     const char* win = row + a.col0 * ELT;
     const int64_t W = a.W;
     const int64_t per = ((W + parts - 1) / parts + VE - 1) / VE * VE;
@@ -1087,38 +1096,32 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
         float pm = wpart[lane].x, ps = wpart[lane].y;
         warp_combine(pm, ps);
         if (lane == 0) {
-            rpart[(int64_t)b * parts + p] = make_float2(pm, ps);
-            __threadfence();
-            s_last = atomicAdd(&a.row_cnt[bk], 1) == parts - 1;
-        }
-    }
-    __syncthreads();
-    if (!s_last) return;
-    // the last piece of the row has arrived: warp 0 combines the pieces in
-    // order while the other warps fetch the root's children's logits
-    __threadfence();
-    if (warp != 0) {
-        for (int32_t i = tid - 32; i < nch; i += ROOT_THREADS - 32)
-            keys[i] = __float_as_uint(load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT));
-    } else {
-        float M = -INFINITY, S = 0.f;
-        for (int base = 0; base < parts; base += 32) {
-            const int g = base + lane;
-            float pm = -INFINITY, ps = 0.f;
-            if (g < parts) {
-                const float2 q = __ldcg(&rpart[(int64_t)b * parts + g]);
-                pm = q.x;
-                ps = q.y;
+            if (parts == 1) {  // the whole row: no pieces to combine
+                s_lse = pm + logf(ps);
+                if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
+            } else {
+                cg::cluster_group cl = cg::this_cluster();
+                cl.map_shared_rank(s_pieces, 0)[p] = make_float2(pm, ps);
             }
-            warp_combine(pm, ps);
-            combine(M, S, pm, ps);
-        }
-        if (lane == 0) {
-            s_lse = M + logf(S);
-            a.row_cnt[bk] = 0;
-            if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
         }
     }
+    if (parts > 1) {
+        cg::this_cluster().sync();  // every piece is in the first CTA's s_pieces
+        if (p != 0) return;
+        if (warp == 0) {
+            float pm = lane < parts ? s_pieces[lane].x : -INFINITY;
+            float ps = lane < parts ? s_pieces[lane].y : 0.f;
+            warp_combine(pm, ps);
+            if (lane == 0) {
+                s_lse = pm + logf(ps);
+                if (!isfinite(s_lse)) set_error(a.err, FR_ERR_NAN_LOGIT);
+            }
+        }
+    }
+    // the root's children's logits, as raw bits until the log-sum-exp is known
+    if (tid < nch) keys[tid] = __float_as_uint(child_x);
+    for (int32_t i = ROOT_THREADS + tid; i < nch; i += ROOT_THREADS)
+        keys[i] = __float_as_uint(load_elem(row, tb + (dense ? i : __ldg(codes + i)), ELT));
     if (tid == 0) {
         s_off[0] = 0;
         s_off[1] = nch;
@@ -1217,7 +1220,6 @@ cudaError_t root_step_setup() {
                                 (int)(ROOT_MAX_CANDS * sizeof(uint32_t)));
 }
 
-int32_t root_step_max_parts() { return ROOT_MAX_PARTS; }
 
 cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, const void* logits,
                              int64_t ld, cudaStream_t s) {
@@ -1263,9 +1265,10 @@ cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const 
     parts = parts < ROOT_MAX_PARTS ? parts : ROOT_MAX_PARTS;
     parts = parts > 1 ? parts : 1;
     if (a.slice_norm) parts = 1;  // nothing is streamed: one CTA per request
-    StepLaunch L(dim3((unsigned)parts, (unsigned)sh.B), ROOT_THREADS, ROOT_MAX_CANDS * sizeof(uint32_t), s);
-    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_root_step<true>, a, sl, parts, buf.root_partial)
-                               : cudaLaunchKernelEx(&L.cfg, k_root_step<false>, a, sl, parts, buf.root_partial);
+    StepLaunch L(dim3((unsigned)parts, (unsigned)sh.B), ROOT_THREADS, ROOT_MAX_CANDS * sizeof(uint32_t), s,
+                 parts > 1 ? (unsigned)parts : 0u);
+    return sh.dtype == FR_BF16 ? cudaLaunchKernelEx(&L.cfg, k_root_step<true>, a, sl, parts)
+                               : cudaLaunchKernelEx(&L.cfg, k_root_step<false>, a, sl, parts);
 }
 
 cudaError_t launch_step_lse(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,

@@ -16,7 +16,6 @@ struct StepBuffers {
     float* cand_key;      // [B * cand_stride] perturbed keys (sampling above temperature 0)
     int64_t cand_stride;  // K * max_fanout rounded up to a multiple of 4
     float2* partial;      // [grid * 2] (max, scaled sum) per CTA and row side
-    float2* root_partial;  // [B * root_step_max_parts()] pieces of the root rows (fused step 0)
     int32_t* row_cnt;     // [B*K] arrival counters of shared rows
     int32_t* err;         // sticky device status word
 };
@@ -88,7 +87,6 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
 // limit (once per device).
 bool root_step_fused(const StepShape& sh, const TrieDev& trie);
 cudaError_t root_step_setup();
-int32_t root_step_max_parts();
 cudaError_t launch_root_step(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, const void* logits,
                              int64_t ld, cudaStream_t s);
 // Log-sum-exp of `rows` rows (row k at logits + k*ld elements) into lse_out,

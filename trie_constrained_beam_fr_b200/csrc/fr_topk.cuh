@@ -494,12 +494,16 @@ __device__ int block_topk(const Vals& vals, int n, int Kp, unsigned long long* o
 // bin's starts; the digit is (key >> s_misc[3]) & s_misc[4]).  s_misc[6] = 1
 // when tmp[0..M) is already in order (every key the same: the Kp lowest slots).
 // Returns -1 when those bins hold more than SORT_CAP keys or one of them more
-// than RANK_CAP.  All threads of the block (blockDim.x == SEL_THREADS) call
-// it; the keys must be readable by all of them on entry; it ends with a
-// barrier.  Scratch: hist [HBINS], tmp [SORT_CAP], red [64], s_misc [8].
+// than RANK_CAP.  digits (shared memory, n entries, or null): the histogram
+// pass records every key's bin there, and the gathering pass then scans the
+// bins instead of the keys, reading only the gathered keys again (for keys in
+// global memory: one full pass fewer).  All threads of the block
+// (blockDim.x == SEL_THREADS) call it; the keys must be readable by all of
+// them on entry; it ends with a barrier.  Scratch: hist [HBINS],
+// tmp [SORT_CAP], red [64], s_misc [8].
 template <class Vals>
 __device__ int block_gather_top(const Vals& vals, int n, int Kp, uint32_t va, uint32_t vo, unsigned long long* tmp,
-                                int32_t* hist, uint32_t* red, int32_t* s_misc) {
+                                int32_t* hist, uint32_t* red, int32_t* s_misc, uint16_t* digits = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = SEL_THREADS / 32;
     reinterpret_cast<int4*>(hist)[tid] = make_int4(0, 0, 0, 0);
@@ -519,7 +523,46 @@ __device__ int block_gather_top(const Vals& vals, int n, int Kp, uint32_t va, ui
     const int lo = 32 - __clz(diff);  // bits >= lo are the same in every key
     const int width = min(HBITS, lo), shift = lo - width;
     const uint32_t dmask = (1u << width) - 1u;
-    for_keys(vals, n, [&](int, uint32_t k) { atomicAdd(&hist[(k >> shift) & dmask], 1); });
+    if (digits) {
+        if constexpr (Vals::QUADS) {  // four bins per 8-byte store
+            const int nq = n >> 2;
+            for (int q0 = tid; q0 < nq; q0 += 8 * SEL_THREADS) {
+                uint4 k4[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int q = q0 + u * SEL_THREADS;
+                    k4[u] = q < nq ? vals.key4(q) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int q = q0 + u * SEL_THREADS;
+                    if (q < nq) {
+                        const uint32_t d0 = (k4[u].x >> shift) & dmask, d1 = (k4[u].y >> shift) & dmask;
+                        const uint32_t d2 = (k4[u].z >> shift) & dmask, d3 = (k4[u].w >> shift) & dmask;
+                        reinterpret_cast<uint2*>(digits)[q] = make_uint2(d0 | (d1 << 16), d2 | (d3 << 16));
+                        atomicAdd(&hist[d0], 1);
+                        atomicAdd(&hist[d1], 1);
+                        atomicAdd(&hist[d2], 1);
+                        atomicAdd(&hist[d3], 1);
+                    }
+                }
+            }
+            const int i = 4 * nq + tid;  // the last n mod 4
+            if (i < n) {
+                const uint32_t d = (vals.key(i) >> shift) & dmask;
+                digits[i] = (uint16_t)d;
+                atomicAdd(&hist[d], 1);
+            }
+        } else {
+            for_keys(vals, n, [&](int i, uint32_t k) {
+                const uint32_t d = (k >> shift) & dmask;
+                digits[i] = (uint16_t)d;
+                atomicAdd(&hist[d], 1);
+            });
+        }
+    } else {
+        for_keys(vals, n, [&](int, uint32_t k) { atomicAdd(&hist[(k >> shift) & dmask], 1); });
+    }
     __syncthreads();
     // keys above each bin: thread t owns bins 4t .. 4t+3, higher threads own
     // higher bins; a scan over the threads from the top
@@ -555,14 +598,24 @@ __device__ int block_gather_top(const Vals& vals, int n, int Kp, uint32_t va, ui
     const int bstar = s_misc[0];
     const int M = s_misc[1] + s_misc[2];
     if (M > SORT_CAP || s_misc[5] != 0) return -1;
-    const uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
-    const uint32_t floor_key = prefix | ((uint32_t)bstar << shift);  // keys >= it: bins >= bstar
-    for_keys(vals, n, [&](int i, uint32_t k) {
-        if (k >= floor_key) {
-            const int p = atomicAdd(&hist[(k >> shift) & dmask], 1);
-            if (p < M) tmp[p] = vals.val_of(i, k);  // always: the keys are the ones counted
+    if (digits) {
+        for (int i = tid; i < n; i += SEL_THREADS) {
+            const int d = digits[i];
+            if (d >= bstar) {
+                const int p = atomicAdd(&hist[d], 1);
+                if (p < M) tmp[p] = vals.val(i);  // always: the keys are the ones counted
+            }
         }
-    });
+    } else {
+        const uint32_t prefix = (lo == 32) ? 0u : (VA & (0xFFFFFFFFu << lo));
+        const uint32_t floor_key = prefix | ((uint32_t)bstar << shift);  // keys >= it: bins >= bstar
+        for_keys(vals, n, [&](int i, uint32_t k) {
+            if (k >= floor_key) {
+                const int p = atomicAdd(&hist[(k >> shift) & dmask], 1);
+                if (p < M) tmp[p] = vals.val_of(i, k);  // always: the keys are the ones counted
+            }
+        });
+    }
     if (tid == 0) {
         s_misc[3] = shift;
         s_misc[4] = (int32_t)dmask;
@@ -577,13 +630,36 @@ __device__ int block_gather_top(const Vals& vals, int n, int Kp, uint32_t va, ui
 // values block_gather_top gathers each go to their bin's first place plus the
 // number of larger values in their bin (at most RANK_CAP comparisons); when it
 // declines, the radix selection (block_topk) finds the winners and they are
-// sorted.  Same calling rules and scratch as block_gather_top.
+// sorted.  At most 64 values: one warp ranks them all.  Same calling rules
+// and scratch as block_gather_top.
 template <class Vals>
 __device__ int block_topk_sorted(const Vals& vals, int n, int Kp, uint32_t va, uint32_t vo, unsigned long long* out,
-                                 unsigned long long* tmp, int32_t* hist, uint32_t* red, int32_t* s_misc) {
+                                 unsigned long long* tmp, int32_t* hist, uint32_t* red, int32_t* s_misc,
+                                 uint16_t* digits = nullptr) {
     const int tid = threadIdx.x;
     if (Kp <= 0 || n <= 0) return 0;
-    const int M = block_gather_top(vals, n, Kp, va, vo, tmp, hist, red, s_misc);
+    if (n <= 64) {
+        // few values: warp 0 ranks all of them (two per lane, each against
+        // every value through shuffles; padding 0 is below every value)
+        __syncthreads();  // the values may have just been written by other warps
+        if (tid < 32) {
+            const unsigned long long v0 = tid < n ? vals.val(tid) : 0ull;
+            const unsigned long long v1 = tid + 32 < n ? vals.val(tid + 32) : 0ull;
+            int r0 = 0, r1 = 0;
+#pragma unroll 1
+            for (int j = 0; j < 32; ++j) {
+                const unsigned long long o0 = __shfl_sync(0xffffffffu, v0, j);
+                const unsigned long long o1 = __shfl_sync(0xffffffffu, v1, j);
+                r0 += (o0 > v0) + (o1 > v0);
+                r1 += (o0 > v1) + (o1 > v1);
+            }
+            if (tid < n && r0 < Kp) out[r0] = v0;
+            if (tid + 32 < n && r1 < Kp) out[r1] = v1;
+        }
+        __syncthreads();
+        return Kp;
+    }
+    const int M = block_gather_top(vals, n, Kp, va, vo, tmp, hist, red, s_misc, digits);
     if (M >= 0) {
         if (s_misc[6]) {
             for (int j = tid; j < Kp; j += SEL_THREADS) out[j] = tmp[j];
