@@ -117,7 +117,8 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     }
     bytes += 2 * align256(sizeof(int32_t) * bk);                   // parent, token
     bytes += 2 * align256(sizeof(float) * (size_t)B * cand_stride);  // cand, cand_key
-    bytes += align256(sizeof(float2) * (size_t)sms * 2);           // partial
+    bytes += align256(sizeof(float2) * (size_t)fr::stream_max_pieces(sms) * 2);  // partial
+    bytes += align256(sizeof(int32_t) * 2);                        // piece_ctr
     bytes += align256(sizeof(int32_t) * bk);                       // row_cnt
     bytes += align256(sizeof(int32_t));                            // err
     cudaError_t e = cudaMalloc(&bm->block, bytes);
@@ -142,7 +143,8 @@ extern "C" fr_status fr_beam_init(const fr_trie* trie, int32_t B, int32_t K, int
     bm->buf.cand = carve<float>(p, (size_t)B * cand_stride);
     bm->buf.cand_key = carve<float>(p, (size_t)B * cand_stride);
     bm->buf.cand_stride = cand_stride;
-    bm->buf.partial = carve<float2>(p, (size_t)sms * 2);
+    bm->buf.partial = carve<float2>(p, (size_t)fr::stream_max_pieces(sms) * 2);
+    bm->buf.piece_ctr = carve<int32_t>(p, 2);
     bm->buf.row_cnt = carve<int32_t>(p, bk);
     bm->buf.err = carve<int32_t>(p, 1);
 

@@ -243,7 +243,11 @@ __global__ void k_reset(StateDev s0, StepBuffers buf, int32_t B, int32_t K, int3
     int32_t root_lo, root_hi;
     trie_children(trie, 0, 0, root_lo, root_hi);
     const int32_t root_fan = root_hi - root_lo;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *buf.err = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *buf.err = 0;
+        buf.piece_ctr[0] = 0;  // after an aborted step the counters may not have been set back
+        buf.piece_ctr[1] = 0;
+    }
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nbk; i += (int64_t)gridDim.x * blockDim.x) {
         const int32_t b = (int32_t)(i / K), k = (int32_t)(i % K);
         const bool root = (k == 0);

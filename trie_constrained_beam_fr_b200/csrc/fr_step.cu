@@ -12,19 +12,27 @@
 //            then, for each row, the trie children's candidate scores
 //            score_k + (x[token] - lse_k).  HBM-bound: the live rows are read
 //            exactly once.  Persistent grid, one CTA per SM.  The flat element
-//            space of all live rows (request-major) is cut into equal,
-//            1024-element-aligned ranges, one per CTA, so every CTA streams
-//            the same number of bytes whatever the row count.  Inside a CTA
-//            one producer lane moves chunks from HBM into a shared-memory
-//            ring (bf16: 5 stages of 40 KB; fp32: 3 of 50 KB) with 1-D bulk
-//            async copies completing on mbarriers; 20 consumer warps each
-//            reduce a lane-interleaved slice of every chunk (running
-//            reference + scaled exp2 sum per lane).  At the end of a
-//            row segment the last consumer warp to arrive combines the 16
-//            warp partials in a fixed order and finishes the row; a row split
-//            across CTAs is finished by the last CTA to arrive (atomic
-//            counter, no waiting) from the per-CTA partials in CTA order.
-//            Ragged heads/tails that are not 16-byte aligned use plain loads.
+//            space of all live rows (request-major) is cut into pieces: one
+//            equal, 1024-element-aligned static piece per CTA over the first
+//            7/8 of the rows, then whole rows that the CTAs take from a
+//            counter as they finish (make_pieces), so that the SMs that
+//            stream faster take more (measured on B200: with equal static
+//            ranges alone the CTAs' ends spread over 13-19 us of a 340-420 us
+//            launch).  Inside a CTA one producer lane schedules: it takes the
+//            pieces, publishes them for the finishers and moves chunks from
+//            HBM into a shared-memory ring (bf16: 5 stages of 40 KB; fp32: 3
+//            of 50 KB) with 1-D bulk async copies completing on mbarriers,
+//            describing each chunk (row, vectors, ragged ends, segment end)
+//            in its stage's metadata; 20 consumer warps each reduce a
+//            lane-interleaved slice of every chunk (running reference +
+//            scaled exp2 sum per lane).  At the end of a row segment the last
+//            consumer warp to arrive combines the 20 warp partials in a fixed
+//            order and queues the row for the two finisher warps, which write
+//            its candidates; a row split across pieces is finished by the
+//            last CTA to arrive (atomic counter, no waiting) from the
+//            per-piece partials in piece order, so the result does not depend
+//            on which CTA took which piece.  Ragged heads/tails that are not
+//            16-byte aligned use plain loads.
 //
 // Above temperature 0 ("flashrec 0.1.1 METADATA", §Serving/API: sampling
 // without replacement by Gumbel perturbation) the candidate writers also store
@@ -80,8 +88,30 @@ static_assert(Ring<true>::STAGES <= MAX_STAGES && Ring<false>::STAGES <= MAX_STA
 constexpr int QCAP = 32;    // finished-segment jobs in flight per CTA
 constexpr int PSLOTS = 32;  // segment-partial slots (segment index mod PSLOTS)
 static_assert(PSLOTS > 2 * MAX_STAGES, "partial slots must outnumber the segments in flight");
-constexpr int64_t GRAN = 1024;  // CTA ranges start at multiples of this many elements
+constexpr int64_t GRAN = 1024;  // pieces start at multiples of this many elements
 constexpr float L2E = 1.4426950408889634f;
+// Pieces of the flat element space (see make_pieces): the first
+// STATIC_NUM / STATIC_DEN of the rows in one static piece per CTA, the other
+// rows in dynamic pieces of whole rows (at most DYN_MAX_PER_CTA per CTA on
+// average) taken from a counter; a CTA's piece list lives in a ring of PCAP
+// entries.
+constexpr int64_t STATIC_NUM = 7, STATIC_DEN = 8;
+constexpr int64_t DYN_MAX_PER_CTA = 32;
+constexpr int PCAP = 64;
+
+// What the producer tells the consumers about the chunk in a ring stage.
+struct StageMeta {
+    const char* ptr;  // the segment's window (its ragged head and tail are read from here)
+    int64_t head_c;   // first unaligned head element (the segment's first chunk), column
+    int64_t tail_c;   // first unaligned tail element (its last chunk), column
+    int64_t r;        // the segment's row
+    int32_t nvec;     // 16-byte vectors in the chunk
+    int32_t head_n;   // unaligned head elements
+    int32_t tail_n;   // unaligned tail elements
+    int32_t jid;      // >= 0: the chunk ends the segment with this job id; -1: more follow
+    int32_t end;      // 1: no chunk; the stream is over
+    int32_t pad;
+};
 
 
 
@@ -98,6 +128,13 @@ struct SmemHdr {
     Job jobs[QCAP];
     int32_t ready[QCAP];  // job id + 1 once jobs[slot] holds that job
     int32_t freed[QCAP];  // job id + 1 once a finisher has copied it out
+    StageMeta meta[MAX_STAGES];  // per ring stage
+    int32_t plist[PCAP];  // this CTA's pieces in order (-1: no more), entry n at n % PCAP
+    int64_t pbeg[PCAP];   // their element ranges [pbeg, pend)
+    int64_t pend[PCAP];
+    int64_t geom[4];      // the launch's piece geometry (Pieces: E, qs, es, qd), set before entry 0
+    int32_t pcount;       // entries published
+    int32_t pfin[NFW];    // pieces each finisher warp has finished
     int32_t abort_flag;
     int32_t pad;
 };
@@ -129,6 +166,8 @@ struct StreamArgs {
     uint64_t wait_ns;    // limit of the bounded waits that give up (abort)
     int32_t starve;      // test setting: the producer issues no copies, so the consumers' waits expire
     int32_t slice_norm;  // fused first step: the log-sum-exp runs over the candidate slice alone
+    int32_t* piece_ctr;  // [2] dynamic pieces taken, CTAs done taking (zero between launches); null:
+                         // static pieces only
 };
 
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the finaliser of a Weyl
@@ -207,6 +246,72 @@ __device__ __forceinline__ bool wait_seq(volatile int32_t* word, int32_t want, v
             return false;
         }
     }
+}
+
+// Bounded wait until *word >= want (a count another warp of this CTA raises).
+__device__ __forceinline__ bool wait_ge(volatile int32_t* word, int32_t want, volatile int32_t* abort_flag,
+                                        int32_t* err, uint64_t limit_ns) {
+    if (*word >= want) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (*word >= want) return true;
+        if (*abort_flag) return false;
+        __nanosleep(64);
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            set_error(err, FR_ERR_DEVICE);
+            return false;
+        }
+    }
+}
+
+// The flat element space [0, E) of a launch's live rows (request-major; E a
+// multiple of the row length W) is cut into pieces.  Without a piece counter:
+// G equal GRAN-aligned pieces, piece p for CTA p.  With one: the first
+// STATIC_NUM / STATIC_DEN of the rows in G equal GRAN-aligned static pieces,
+// CTA p's own, then the remaining rows in dynamic pieces of whole rows that
+// the CTAs take from the counter as they finish their previous piece, so that
+// CTAs on SMs that stream faster take more and all of them end within about
+// one row of each other.  A dynamic row is never split, so it is finished by
+// the CTA that streamed it.  The boundaries depend only on E, W and G: a
+// row's partial sums are combined the same way whichever CTA reduces each
+// piece.
+struct Pieces {
+    int64_t E, qs, es, qd;  // qs elements per static piece, es = G * qs, qd per dynamic piece
+    int32_t G, np;          // CTAs, pieces in all
+};
+__device__ __forceinline__ Pieces make_pieces(int64_t E, int32_t G, int64_t W, bool dyn) {
+    Pieces P;
+    P.E = E;
+    P.G = G;
+    if (!dyn) {
+        P.qs = ((E + G - 1) / G + GRAN - 1) / GRAN * GRAN;
+        P.es = E;
+        P.qd = W;
+        P.np = G;
+        return P;
+    }
+    // whole rows: the last (1 - STATIC_NUM / STATIC_DEN) of them, in pieces
+    // of qd / W rows, are dynamic
+    const int64_t rows = E / W;
+    const int64_t srows = rows * STATIC_NUM / STATIC_DEN;
+    P.es = srows * W;
+    P.qs = ((P.es + G - 1) / G + GRAN - 1) / GRAN * GRAN;
+    const int64_t drows = rows - srows;
+    const int64_t cap = (int64_t)G * DYN_MAX_PER_CTA;
+    const int64_t k = (drows + cap - 1) / cap > 1 ? (drows + cap - 1) / cap : 1;
+    P.qd = k * W;
+    P.np = G + (int32_t)((drows + k - 1) / k);
+    return P;
+}
+__device__ __forceinline__ int64_t piece_begin(const Pieces& P, int64_t p) {
+    return p < P.G ? min(P.es, p * P.qs) : min(P.E, P.es + (p - P.G) * P.qd);
+}
+__device__ __forceinline__ int64_t piece_end(const Pieces& P, int64_t p) {
+    return p < P.G ? min(P.es, (p + 1) * P.qs) : min(P.E, P.es + (p - P.G + 1) * P.qd);
+}
+__device__ __forceinline__ int64_t piece_of(const Pieces& P, int64_t e) {
+    return e < P.es ? e / P.qs : P.G + (e - P.es) / P.qd;
 }
 
 __device__ __forceinline__ int find_request(const int32_t* row_start, int B, int64_t r) {
@@ -543,19 +648,33 @@ __device__ __forceinline__ void finish_row(const StreamArgs& a, const Seg& sg, f
 }
 
 // Called by the warp that combined this CTA's partial for row r.
-__device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, int64_t r_first, int64_t Q, float m,
-                               float s, const RowPrep& p) {
+__device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, const int64_t* geom, int64_t piece,
+                               float m, float s, const RowPrep& p) {
     const int lane = threadIdx.x & 31;
-    const int64_t fc = (r * a.W) / Q;
-    const int64_t lc = ((r + 1) * a.W - 1) / Q;
+    int64_t fc, lc, beg_fc, beg_piece;
+    {
+        Pieces P;  // as the producer made it
+        P.E = geom[0];
+        P.qs = geom[1];
+        P.es = geom[2];
+        P.qd = geom[3];
+        P.G = (int32_t)gridDim.x;
+        fc = piece_of(P, r * a.W);
+        lc = piece_of(P, (r + 1) * a.W - 1);
+        beg_fc = piece_begin(P, fc);
+        beg_piece = piece_begin(P, piece);
+    }
     if (fc == lc) {
         finish_row(a, sg, m, s, p);
         return;
     }
-    const int side = (r == r_first) ? 0 : 1;
+    // a piece's partial of its first row is in its slot 0, of its last in
+    // slot 1: here slot 1 only for the first piece, when it starts before r
+    const int64_t rs = r * a.W;
+    const int side = beg_piece >= rs ? 0 : 1;
     int old = 0;
     if (lane == 0) {
-        a.partial[(int64_t)blockIdx.x * 2 + side] = make_float2(m, s);
+        a.partial[piece * 2 + side] = make_float2(m, s);
         __threadfence();
         old = atomicAdd(&a.row_cnt[r], 1);
     }
@@ -567,10 +686,10 @@ __device__ void finish_segment(const StreamArgs& a, const Seg& sg, int64_t r, in
         const int64_t gg = base + lane;
         float pm = -INFINITY, ps = 0.f;
         if (gg <= lc) {
-            const int sd = ((gg * Q) / a.W == r) ? 0 : 1;
-            const float2 p = __ldcg(&a.partial[gg * 2 + sd]);
-            pm = p.x;
-            ps = p.y;
+            const int sd = (gg == fc && beg_fc < rs) ? 1 : 0;
+            const float2 q = __ldcg(&a.partial[gg * 2 + sd]);
+            pm = q.x;
+            ps = q.y;
         }
         warp_combine(pm, ps);
         combine(M, S, pm, ps);
@@ -621,6 +740,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
             hdr->freed[i] = 0;
         }
         for (int i = lane; i < PSLOTS; i += 32) hdr->segcnt[i] = 0;
+        if (lane < NFW) hdr->pfin[lane] = 0;
+        if (lane == 0) hdr->pcount = 0;
         if (lane == 0) {
             for (int i = 0; i < STAGES; ++i) {
                 mbar_init(&hdr->full[i], 1);
@@ -634,43 +755,100 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
 
     const int64_t E = (int64_t)row_start[a.B] * a.W;
     if (E == 0) return;
-    const int64_t G = gridDim.x;
-    const int64_t Q = ((E + G - 1) / G + GRAN - 1) / GRAN * GRAN;
-    const int64_t bg = min(E, (int64_t)blockIdx.x * Q);
-    const int64_t eg = min(E, (int64_t)(blockIdx.x + 1) * Q);
-    if (bg >= eg) return;
-    const int64_t r_first = bg / a.W, r_last = (eg - 1) / a.W;
 
     if (warp == PRODUCER_WARP) {
+        // The producer lane is the CTA's scheduler: it takes the pieces (its
+        // own static piece, then dynamic ones from the counter), publishes
+        // each in the piece list (for the finishers) before streaming it,
+        // and describes every chunk in its stage's StageMeta (for the
+        // consumers); a last, empty stage with `end` set closes the stream.
         if (lane == 0 && !a.starve) {
+            const Pieces P = make_pieces(E, (int32_t)gridDim.x, a.W, a.piece_ctr != nullptr);
+            hdr->geom[0] = P.E;
+            hdr->geom[1] = P.qs;
+            hdr->geom[2] = P.es;
+            hdr->geom[3] = P.qd;
             uint32_t chunk = 0;
             int st = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int64_t r = r_first; r <= r_last && ok; ++r) {
-                const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
-                const char* src = sg.ptr + sg.a0 * ELT;
-                int64_t left = (sg.a1 - sg.a0) * ELT;
-                for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
+            int32_t jid = 0;
+            int64_t pc = blockIdx.x;
+            for (int32_t n = 0; ok; ++n) {
+                if (pc >= P.np) pc = -1;
+                if (n >= PCAP) {  // entry n - PCAP must be done with
+#pragma unroll
+                    for (int f = 0; f < NFW; ++f)
+                        if (ok && !wait_ge(&hdr->pfin[f], n - PCAP + 1, &hdr->abort_flag, a.err, a.wait_ns)) ok = false;
+                    if (!ok) break;
+                }
+                const int64_t bg = pc < 0 ? 0 : piece_begin(P, pc), eg = pc < 0 ? 0 : piece_end(P, pc);
+                hdr->plist[n % PCAP] = (int32_t)pc;
+                hdr->pbeg[n % PCAP] = bg;
+                hdr->pend[n % PCAP] = eg;
+                __threadfence_block();
+                *(volatile int32_t*)&hdr->pcount = n + 1;
+                if (pc < 0) {
+                    // close the stream: one more stage, with no chunk
                     if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err, a.wait_ns)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t bytes =
-                        (uint32_t)(left < (int64_t)STAGE_BYTES ? (left > 0 ? left : 0) : STAGE_BYTES);
-                    if (bytes) {
-                        mbar_arrive_expect_tx(&hdr->full[st], bytes);
-                        bulk_g2s(ring + (size_t)st * STAGE_BYTES, src, bytes, &hdr->full[st]);
-                    } else {
-                        mbar_arrive(&hdr->full[st]);
+                    hdr->meta[st].end = 1;
+                    mbar_arrive(&hdr->full[st]);
+                    break;
+                }
+                int64_t nxt = P.np;
+                bool asked = a.piece_ctr == nullptr;
+                const int64_t r_last = bg < eg ? (eg - 1) / a.W : -1;
+                for (int64_t r = bg / a.W; r <= r_last && ok; ++r, ++jid) {
+                    if (r == r_last && !asked) {  // the next piece, asked for a row ahead
+                        nxt = (int64_t)P.G + atomicAdd(a.piece_ctr, 1);
+                        asked = true;
                     }
-                    src += STAGE_BYTES;
-                    left -= STAGE_BYTES;
-                    if (++st == STAGES) {
-                        st = 0;
-                        ph ^= 1u;
+                    const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
+                    const char* src = sg.ptr + sg.a0 * ELT;
+                    int64_t left = (sg.a1 - sg.a0) * ELT;
+                    const int32_t nvec_all = (int32_t)((sg.a1 - sg.a0) * ELT / 16);
+                    for (int j = 0; j < sg.nchunks; ++j, ++chunk) {
+                        if (!wait_bar(&hdr->empty[st], ph ^ 1u, &hdr->abort_flag, a.err, a.wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        StageMeta& mt = hdr->meta[st];
+                        mt.ptr = sg.ptr;
+                        mt.head_c = sg.c0;
+                        mt.tail_c = sg.a1;
+                        mt.r = r;
+                        mt.nvec = min(nvec_all - j * VEC_PER_STAGE, VEC_PER_STAGE);
+                        mt.head_n = (j == 0) ? (int32_t)(sg.a0 - sg.c0) : 0;
+                        mt.tail_n = (j == sg.nchunks - 1) ? (int32_t)(sg.c1 - sg.a1) : 0;
+                        mt.jid = (j == sg.nchunks - 1) ? jid : -1;
+                        mt.end = 0;
+                        const uint32_t bytes =
+                            (uint32_t)(left < (int64_t)STAGE_BYTES ? (left > 0 ? left : 0) : STAGE_BYTES);
+                        if (bytes) {
+                            mbar_arrive_expect_tx(&hdr->full[st], bytes);
+                            bulk_g2s(ring + (size_t)st * STAGE_BYTES, src, bytes, &hdr->full[st]);
+                        } else {
+                            mbar_arrive(&hdr->full[st]);
+                        }
+                        src += STAGE_BYTES;
+                        left -= STAGE_BYTES;
+                        if (++st == STAGES) {
+                            st = 0;
+                            ph ^= 1u;
+                        }
                     }
                 }
+                if (!asked && ok) nxt = (int64_t)P.G + atomicAdd(a.piece_ctr, 1);  // an empty piece
+                pc = nxt;
+            }
+            // the last CTA to be done taking pieces sets the counter back for
+            // the next launch
+            if (a.piece_ctr && atomicAdd(a.piece_ctr + 1, 1) == (int)gridDim.x - 1) {
+                a.piece_ctr[0] = 0;
+                a.piece_ctr[1] = 0;
             }
             if (!ok) {
                 const uint32_t first = chunk > (uint32_t)STAGES ? chunk - STAGES : 0u;
@@ -681,107 +859,123 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1) k_stream(const StreamArgs a
     }
 
     if (warp >= FIRST_FINISHER_WARP) {
-        // Finishers take the reduced segments in order (job j = row r_first + j)
-        // from the queue the consumers fill, so that the gathers of the
-        // candidate scores never hold up the ring.
-        const int64_t njobs = r_last - r_first + 1;
-        for (int64_t j = warp - FIRST_FINISHER_WARP; j < njobs; j += NFW) {
-            const int slot = (int)(j % QCAP);
-            const int64_t r = r_first + j;
-            const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
-            const RowPrep prep = prep_cands(a, sg);  // while row r streams
-            if (!wait_seq(&hdr->ready[slot], (int32_t)(j + 1), &hdr->abort_flag, a.err, a.wait_ns)) return;
+        // Finishers take the reduced segments in order (job g: the g-th row
+        // segment of this CTA, over its pieces in list order; finisher warp
+        // g % NFW) from the queue the consumers fill, so that the gathers of
+        // the candidate scores never hold up the ring.
+        const int fw = warp - FIRST_FINISHER_WARP;
+        int32_t jbase = 0;
+        for (int32_t n = 0;; ++n) {
+            if (!wait_ge(&hdr->pcount, n + 1, &hdr->abort_flag, a.err, a.wait_ns)) return;
             __threadfence_block();
-            const Job job = hdr->jobs[slot];
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(j + 1);
+            const int32_t pc = hdr->plist[n % PCAP];
+            if (pc < 0) break;
+            const int64_t bg = hdr->pbeg[n % PCAP], eg = hdr->pend[n % PCAP];
+            if (bg < eg) {
+                const int64_t r_first = bg / a.W;
+                const int32_t njobs = (int32_t)((eg - 1) / a.W - r_first + 1);
+                for (int32_t j = (fw - jbase % NFW + NFW) % NFW; j < njobs; j += NFW) {
+                    const int32_t g = jbase + j;
+                    const int slot = (int)(g % QCAP);
+                    const int64_t r = r_first + j;
+                    const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
+                    const RowPrep prep = prep_cands(a, sg);  // while row r streams
+                    if (!wait_seq(&hdr->ready[slot], (int32_t)(g + 1), &hdr->abort_flag, a.err, a.wait_ns)) return;
+                    __threadfence_block();
+                    const Job job = hdr->jobs[slot];
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence_block();
+                        *(volatile int32_t*)&hdr->freed[slot] = (int32_t)(g + 1);
+                    }
+                    finish_segment(a, sg, r, hdr->geom, pc, job.m, job.s, prep);
+                }
+                jbase += njobs;
             }
-            finish_segment(a, sg, r, r_first, Q, job.m, job.s, prep);
+            __syncwarp();
+            if (lane == 0) *(volatile int32_t*)&hdr->pfin[fw] = n + 1;
         }
         return;
     }
 
-    // consumers: every warp reduces its lane-interleaved share of each chunk
+    // consumers: every warp reduces its lane-interleaved share of each chunk,
+    // as the stage's StageMeta describes it
     const int cw = warp;
     const int vbase = cw * 32 + lane;
     int st = 0;
     uint32_t ph = 0;
     float m = -INFINITY;
     f32x2 s2 = pack2(0.f, 0.f);
-    for (int64_t r = r_first; r <= r_last; ++r) {
-        const Seg sg = make_seg<ELT>(a, row_start, r, bg, eg);
-        const int32_t nvec_all = (int32_t)((sg.a1 - sg.a0) * ELT / 16);
-        for (int j = 0; j < sg.nchunks; ++j) {
-            if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err, a.wait_ns)) return;
-            if (j == 0 && cw == 0 && lane < sg.a0 - sg.c0) lane_add(m, s2, load_elem(sg.ptr, sg.c0 + lane, ELT));
-            const uint4* stage = reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES);
-            const int32_t nvec = min(nvec_all - j * VEC_PER_STAGE, VEC_PER_STAGE);
-            uint4 q[VPL];
-            if (nvec == VEC_PER_STAGE) {
+    for (;;) {
+        if (!wait_bar(&hdr->full[st], ph, &hdr->abort_flag, a.err, a.wait_ns)) return;
+        const StageMeta* mt = &hdr->meta[st];
+        if (mt->end) break;
+        if (cw == 0 && lane < mt->head_n) lane_add(m, s2, load_elem(mt->ptr, mt->head_c + lane, ELT));
+        const uint4* stage = reinterpret_cast<const uint4*>(ring + (size_t)st * STAGE_BYTES);
+        const int32_t nvec = mt->nvec;
+        uint4 q[VPL];
+        if (nvec == VEC_PER_STAGE) {
 #pragma unroll
-                for (int v = 0; v < VPL; ++v) q[v] = stage[vbase + v * (NCW * 32)];
-                lane_consume<BF16>(q, m, s2);
-            } else if (nvec > 0) {
-                constexpr uint32_t NEG = BF16 ? 0xFF80FF80u : 0xFF800000u;
+            for (int v = 0; v < VPL; ++v) q[v] = stage[vbase + v * (NCW * 32)];
+            lane_consume<BF16>(q, m, s2);
+        } else if (nvec > 0) {
+            constexpr uint32_t NEG = BF16 ? 0xFF80FF80u : 0xFF800000u;
 #pragma unroll
-                for (int v = 0; v < VPL; ++v) {
-                    const int idx = vbase + v * (NCW * 32);
-                    q[v] = idx < nvec ? stage[idx] : make_uint4(NEG, NEG, NEG, NEG);
-                }
-                lane_consume<BF16>(q, m, s2);
+            for (int v = 0; v < VPL; ++v) {
+                const int idx = vbase + v * (NCW * 32);
+                q[v] = idx < nvec ? stage[idx] : make_uint4(NEG, NEG, NEG, NEG);
             }
-            const bool last = (j == sg.nchunks - 1);
-            if (last && cw == 0 && lane < sg.c1 - sg.a1) lane_add(m, s2, load_elem(sg.ptr, sg.a1 + lane, ELT));
-            const int cur = st;
-            if (++st == STAGES) {
-                st = 0;
-                ph ^= 1u;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&hdr->empty[cur]);
-            if (!last) continue;
-            // end of this CTA's segment of row r: the last warp to get here
-            // combines the per-warp partials in warp order and queues the job
-            const int64_t jid = r - r_first;
-            const int ps = (int)(jid % PSLOTS);
-            float lo, hi;
-            unpack2(s2, lo, hi);
-            float sum = lo + hi;
-            warp_combine(m, sum);
-            if (lane == 0) hdr->part[ps][cw] = make_float2(m, sum);
-            __syncwarp();
-            int old = 0;
-            if (lane == 0) {
-                __threadfence_block();
-                old = atomicAdd(&hdr->segcnt[ps], 1);
-            }
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if (old == NCW - 1) {
-                __threadfence_block();
-                float pm = -INFINITY, pv = 0.f;
-                if (lane < NCW) {
-                    pm = hdr->part[ps][lane].x;
-                    pv = hdr->part[ps][lane].y;
-                }
-                warp_combine(pm, pv);
-                __syncwarp();
-                if (lane == 0) hdr->segcnt[ps] = 0;
-                const int slot = (int)(jid % QCAP);
-                if (jid >= QCAP &&
-                    !wait_seq(&hdr->freed[slot], (int32_t)(jid - QCAP + 1), &hdr->abort_flag, a.err, a.wait_ns))
-                    return;
-                if (lane == 0) {
-                    hdr->jobs[slot] = Job{r, pm, pv};
-                    __threadfence_block();
-                    *(volatile int32_t*)&hdr->ready[slot] = (int32_t)(jid + 1);
-                }
-                __syncwarp();
-            }
-            m = -INFINITY;
-            s2 = pack2(0.f, 0.f);
+            lane_consume<BF16>(q, m, s2);
         }
+        if (cw == 0 && lane < mt->tail_n) lane_add(m, s2, load_elem(mt->ptr, mt->tail_c + lane, ELT));
+        const int32_t jid = mt->jid;
+        const int64_t r = mt->r;
+        const int cur = st;
+        if (++st == STAGES) {
+            st = 0;
+            ph ^= 1u;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&hdr->empty[cur]);
+        if (jid < 0) continue;
+        // end of this CTA's segment of row r: the last warp to get here
+        // combines the per-warp partials in warp order and queues the job
+        const int ps = (int)(jid % PSLOTS);
+        float lo, hi;
+        unpack2(s2, lo, hi);
+        float sum = lo + hi;
+        warp_combine(m, sum);
+        if (lane == 0) hdr->part[ps][cw] = make_float2(m, sum);
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            old = atomicAdd(&hdr->segcnt[ps], 1);
+        }
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == NCW - 1) {
+            __threadfence_block();
+            float pm = -INFINITY, pv = 0.f;
+            if (lane < NCW) {
+                pm = hdr->part[ps][lane].x;
+                pv = hdr->part[ps][lane].y;
+            }
+            warp_combine(pm, pv);
+            __syncwarp();
+            if (lane == 0) hdr->segcnt[ps] = 0;
+            const int slot = (int)(jid % QCAP);
+            if (jid >= QCAP &&
+                !wait_seq(&hdr->freed[slot], (int32_t)(jid - QCAP + 1), &hdr->abort_flag, a.err, a.wait_ns))
+                return;
+            if (lane == 0) {
+                hdr->jobs[slot] = Job{r, pm, pv};
+                __threadfence_block();
+                *(volatile int32_t*)&hdr->ready[slot] = (int32_t)(jid + 1);
+            }
+            __syncwarp();
+        }
+        m = -INFINITY;
+        s2 = pack2(0.f, 0.f);
     }
 }
 
@@ -1147,6 +1341,8 @@ __global__ void __launch_bounds__(ROOT_THREADS, 1)
 
 }  // namespace
 
+int64_t stream_max_pieces(int32_t grid) { return (int64_t)grid * (1 + DYN_MAX_PER_CTA) + 1; }
+
 size_t stream_smem_bytes(int32_t B, bool bf16) {
     return (size_t)(bf16 ? Ring<true>::RING_BYTES : Ring<false>::RING_BYTES) + sizeof(SmemHdr) +
            sizeof(int32_t) * (size_t)(B + 1);
@@ -1190,6 +1386,7 @@ cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const Tri
     a.req_offset = sh.req_offset;
     a.wait_ns = sh.wait_ns ? sh.wait_ns : FR_WAIT_LIMIT_NS;
     a.starve = sh.starve;
+    a.piece_ctr = buf.piece_ctr;
     a.row_stride_b = sh.K;
     a.col_sub = 0;
     a.lse_in = nullptr;

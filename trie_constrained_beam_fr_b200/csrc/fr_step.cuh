@@ -15,7 +15,8 @@ struct StepBuffers {
     float* cand;          // [B * cand_stride] candidate scores
     float* cand_key;      // [B * cand_stride] perturbed keys (sampling above temperature 0)
     int64_t cand_stride;  // K * max_fanout rounded up to a multiple of 4
-    float2* partial;      // [grid * 2] (max, scaled sum) per CTA and row side
+    float2* partial;      // [stream_max_pieces(grid) * 2] (max, scaled sum) per piece and row side
+    int32_t* piece_ctr;   // [2] the streaming kernel's dynamic-piece counters (zero between launches)
     int32_t* row_cnt;     // [B*K] arrival counters of shared rows
     int32_t* err;         // sticky device status word
 };
@@ -78,6 +79,9 @@ cudaError_t select_kernel_setup();  // raises the one-CTA selection's shared-mem
 // fp32 rows: the ring differs).
 size_t stream_smem_bytes(int32_t B, bool bf16);
 cudaError_t stream_kernel_setup();  // raises the kernel's shared-memory limit
+// Most pieces the streaming kernel cuts a launch into on `grid` CTAs (its
+// partial buffer holds two entries per piece).
+int64_t stream_max_pieces(int32_t grid);
 
 cudaError_t launch_stream(const StepShape& sh, const StepBuffers& buf, const TrieDev& trie, int t,
                           const void* logits, int64_t ld, cudaStream_t s);
