@@ -528,14 +528,20 @@ __device__ __forceinline__ void lane_add(float& m, f32x2& s2, float x) {
 // A row's candidate writer needs, besides the row's log-sum-exp, the beam's
 // running score, its trie children and its candidate offset, and the
 // children's logits.  None of these depends on the reduction, so the finisher
-// loads them (and the first batch of the children's logits: lane l holds
-// children l, l + 32, ..., l + 32 (GATHER - 1)) before it waits for the row,
-// while the row is still streaming; only the rest of the gathers, for rows
-// with more than 32 * GATHER children, come after.
+// loads them (and the first batch of the children's logits) before it waits
+// for the row, while the row is still streaming; only the rest, for rows with
+// many children, comes after.  Children of a dense level are consecutive
+// tokens: when their logits and their candidate run both start on 16 bytes,
+// the writer moves 16-byte groups (8 bf16 or 4 fp32 logits in, as many scores
+// out; lane l's first group prefetched), which at 1,024 children per row
+// keeps the two finisher warps ahead of the stream (measured on B200, narrow
+// step 1: 347 -> 331 us); otherwise lane l gathers children l, l + 32, ...,
+// l + 32 (GATHER - 1) first, one logit at a time.
 constexpr int GATHER = 8;  // independent gathers in flight per lane
 struct RowPrep {
     float sc;
     int32_t lo, nch, base;  // nch < 0: the beam's node or offsets are out of range
+    int32_t vec;            // the 16-byte path (see prep_cands); x[0..3] hold lane's first group
     float x[GATHER];
 };
 
@@ -544,6 +550,7 @@ __device__ __forceinline__ RowPrep prep_cands(const StreamArgs& a, const Seg& sg
     p.sc = 0.f;
     p.lo = p.base = 0;
     p.nch = -1;
+    p.vec = 0;
 #pragma unroll
     for (int u = 0; u < GATHER; ++u) p.x[u] = 0.f;
     if (a.lse_out) return p;  // log-sum-exps only: no candidates
@@ -563,12 +570,51 @@ __device__ __forceinline__ RowPrep prep_cands(const StreamArgs& a, const Seg& sg
     const int32_t* codes = a.trie.code[t + 1] + lo;
     const bool dense = a.trie.dense_c[t] != 0;  // children's codes are 0 .. C-1
     const int32_t tb = a.trie.tok_base[t] - a.col_sub;
+    // dense children (consecutive tokens) whose first logit starts on a
+    // 16-byte boundary and whose candidate run does too: whole 16-byte groups
+    // of logits in, 16-byte groups of scores out (lane l: group l first)
+    const char* first = sg.row + (int64_t)tb * a.elt;
+    if (dense && !a.cand_key && ((reinterpret_cast<uintptr_t>(first) & 15u) == 0) && ((base & 3) == 0)) {
+        p.vec = 1;
+        const int32_t ve = 16 / a.elt;
+        if ((lane + 1) * ve <= p.nch) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(first) + lane);
+            p.x[0] = __uint_as_float(q.x);
+            p.x[1] = __uint_as_float(q.y);
+            p.x[2] = __uint_as_float(q.z);
+            p.x[3] = __uint_as_float(q.w);
+        }
+        return p;
+    }
 #pragma unroll
     for (int u = 0; u < GATHER; ++u) {
         const int32_t i = u * 32 + lane;
         if (i < p.nch) p.x[u] = load_elem(sg.row, tb + (dense ? i : __ldg(codes + i)), a.elt);
     }
     return p;
+}
+
+// Scores of one 16-byte group of logits (8 bf16 or 4 fp32) into out (16-byte
+// aligned).
+__device__ __forceinline__ void write_group(const uint4 q, bool bf16, float sc, float lse, float* out) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    if (bf16) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[2 * e] = sc + (__uint_as_float(w[e] << 16) - lse);
+            v[2 * e + 1] = sc + (__uint_as_float(w[e] & 0xFFFF0000u) - lse);
+        }
+        reinterpret_cast<float4*>(out)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(out)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[e] = sc + (__uint_as_float(w[e]) - lse);
+        }
+        reinterpret_cast<float4*>(out)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    }
 }
 
 // The row's log-sum-exp is known: write the scores of the trie children of
@@ -590,6 +636,30 @@ __device__ void finish_cands(const StreamArgs& a, const Seg& sg, float lse, cons
     const int32_t tb = a.trie.tok_base[t];
     float* out = a.cand + (int64_t)sg.b * a.cand_stride + p.base;
     const int32_t nch = p.nch;
+    if (p.vec) {
+        const bool bf16 = a.elt == 2;
+        const int32_t ve = bf16 ? 8 : 4;
+        const int32_t ng = nch / ve;  // whole groups; the rest one by one
+        const uint4* src = reinterpret_cast<const uint4*>(sg.row + (int64_t)(tb - a.col_sub) * a.elt);
+        for (int32_t g0 = 0; g0 < ng; g0 += 4 * 32) {
+            uint4 q[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int32_t g = g0 + u * 32 + lane;
+                q[u] = (g < ng && g >= 32) ? __ldg(src + g) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (g0 == 0)
+                q[0] = make_uint4(__float_as_uint(p.x[0]), __float_as_uint(p.x[1]), __float_as_uint(p.x[2]),
+                                  __float_as_uint(p.x[3]));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int32_t g = g0 + u * 32 + lane;
+                if (g < ng) write_group(q[u], bf16, sc, lse, out + (int64_t)g * ve);
+            }
+        }
+        for (int32_t i = ng * ve + lane; i < nch; i += 32) out[i] = sc + (load_elem(sg.row, tb + i - a.col_sub, a.elt) - lse);
+        return;
+    }
     if (a.cand_key) {
         float* key = a.cand_key + (int64_t)sg.b * a.cand_stride + p.base;
         const uint64_t rh = gumbel_row_hash(a.gseed, a.req_offset + sg.b, t);
